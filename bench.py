@@ -1,0 +1,394 @@
+"""Benchmark of the MoE layer with zero-computation experts on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
+                    [--impl reference]
+
+One step = one pass of the whole layer (router + top-k, dispatch, grouped
+SwiGLU expert GEMMs, combine) over one batch of seeded synthetic tokens. The
+default workload is the bf16 decode layer (T=64, d=4096, 128 routed experts of
+width 1024 + 32 zero experts, top-8, fp32 router). Prints one JSON line.
+
+Under torchrun each rank runs its own replica on its own batch (seed + rank):
+the layer is data-parallel over tokens with no exchange, so scaling is weak
+and the only collectives are the timing barrier and the max over ranks.
+
+``--impl reference`` times the CPU oracle (fp64, OpenMP) on a bounded sample
+of the same workload on this machine's host cores; rank 0 only.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from moe_synth import get_config, make_inputs, torch_dtype  # noqa: E402
+
+METRIC = "MoE-layer tokens/s; grouped-GEMM % bf16 TC peak; router/dispatch/combine GB/s"
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return {"hbm_gbs": float(j["hbm_gbs"]), "bf16_tflops": float(j["bf16_tflops"]),
+                "bf16_tflops_sustained": float(j.get("bf16_tflops_sustained", j["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def workload_name(sh):
+    return (f"{sh.name}: T={sh.T}, d={sh.d}, {sh.n_routed} routed experts (SwiGLU, "
+            f"F={sh.ffn}) + {sh.n_zero} zero experts, top-{sh.top_k}, "
+            f"{sh.act_dtype} activations/weights, fp32 router, routing={sh.routing}")
+
+
+# ------------------------------------------------------------------ clocks --
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.t.join(timeout=5)
+        sms, maxs, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for _, line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sms.append(float(parts[1]))
+                maxs.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sms:
+            return None
+        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": max(maxs),
+                "reasons": sorted(reasons), "samples": len(sms)}
+
+
+# --------------------------------------------------------- reference (CPU) --
+def run_reference(args, sh):
+    import oracle
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    inp = make_inputs(sh, args.seed)
+    sample = min(sh.T, args.ref_tokens)
+    toks = torch.arange(sample, dtype=torch.int32).numpy()
+    cores = oracle.num_threads()
+
+    def step():
+        oracle.layer(inp.x, inp.w_router, inp.bias, inp.w_gate, inp.w_up, inp.w_down,
+                     sh.n_routed, sh.top_k, sh.routed_scale, tokens=toks)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    value = args.steps * sample / dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_name(sh), "seed": args.seed},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores,
+                         "kind": "oracle",
+                         "sample": f"per step: whole layer on the first {sample} of "
+                                   f"{sh.T} tokens (fp64 oracle, OpenMP)"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def cpu_baseline(sh, inp, budget_s=12.0):
+    """The oracle, as it stands, on this host's cores: whole layer over the
+    batch, repeated until about budget_s seconds of CPU work."""
+    import oracle
+    cores = oracle.num_threads()
+    n_tok = sh.T if sh.T <= 256 else 256
+    toks = torch.arange(n_tok, dtype=torch.int32).numpy()
+    done, t0 = 0, time.perf_counter()
+    while True:
+        oracle.layer(inp.x, inp.w_router, inp.bias, inp.w_gate, inp.w_up, inp.w_down,
+                     sh.n_routed, sh.top_k, sh.routed_scale, tokens=toks)
+        done += n_tok
+        if time.perf_counter() - t0 >= budget_s or done >= 64 * n_tok:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": done / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"whole layer (fp64) on {n_tok} of {sh.T} tokens, repeated "
+                      f"{done // n_tok}x ({dt:.1f} s)"}
+
+
+# -------------------------------------------------------------- GPU path --
+def graph_time_ms(fn, reps):
+    """Device time per call of fn, captured `reps` times in one CUDA graph so
+    host launch overhead does not hide the kernels' own duration."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        fn()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(reps):
+            fn()
+    g.replay()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    g.replay()
+    end.record(stream)
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(end) / reps
+    del g
+    return ms
+
+
+def event_time_ms(fn, reps, stream):
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(reps):
+        fn()
+    end.record(stream)
+    torch.cuda.synchronize()
+    return start.elapsed_time(end) / reps
+
+
+def run_gpu(args, sh):
+    import expert_routing_dispatch_router_b200 as moe
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+    pk = peaks()
+
+    inp = make_inputs(sh, args.seed + rank)
+    d = inp.to(dev)
+    ls = moe.LayerShape(sh.T, sh.d, sh.n_routed, sh.n_zero, sh.top_k, sh.ffn,
+                        torch_dtype(sh.act_dtype), sh.routed_scale)
+    ws = moe.alloc_workspace(ls, dev)
+    out = torch.empty(sh.T, sh.d, dtype=d.x.dtype, device=dev)
+    counts = torch.empty(sh.E, dtype=torch.int32, device=dev)
+
+    def step():
+        moe.layer_forward(ls, d.x, d.w_router, d.bias, d.w_gate, d.w_up, d.w_down, ws,
+                          out=out, counts=counts)
+
+    step()
+    torch.cuda.synchronize()
+    err = moe.read_device_error(ws)
+    if err != 0:
+        raise RuntimeError(f"device error {err} in the first step")
+    c = counts.cpu()
+    R = int(c[: sh.n_routed].sum())
+    U = int((c[: sh.n_routed] > 0).sum())
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    # warm-up: W steps, and at least ~1.5 s so the clock sampler sees load
+    t_end = time.time() + 1.5
+    n = 0
+    while n < args.warmup or time.time() < t_end:
+        step()
+        n += 1
+        if n % 64 == 0:
+            torch.cuda.synchronize()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(args.steps):
+        step()
+    end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ms = start.elapsed_time(end)
+    if world > 1:
+        tt = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    ms_per_step = ms / args.steps
+    value = world * args.steps * sh.T / (ms / 1e3)
+
+    # ---- end to end through the host-buffer entry point
+    x_host = inp.x.clone().pin_memory()
+    out_host = torch.empty(sh.T, sh.d, dtype=d.x.dtype).pin_memory()
+
+    def step_host():
+        moe.layer_forward_host(ls, x_host, d.w_router, d.bias, d.w_gate, d.w_up, d.w_down,
+                               ws, out_host)
+
+    for _ in range(max(args.warmup, 3)):
+        step_host()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e2e_ms = event_time_ms(step_host, args.steps, stream)
+    if world > 1:
+        tt = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    assert torch.equal(out_host, out.cpu()), "host entry point disagrees with device entry point"
+    act_b = sh.T * sh.d * d.x.element_size()
+
+    # ---- per-stage timings (staged calls, same inputs), rank 0 only
+    comp = {}
+    roof = None
+    if rank == 0:
+        reps = 50
+        idx, gate = moe.route(ls, d.x, d.w_router, d.bias, ws)
+        t_route = graph_time_ms(lambda: moe.route(ls, d.x, d.w_router, d.bias, ws), reps)
+        cnt, offs, row_tok, slot_row, x_perm = moe.dispatch(ls, d.x, idx, ws)
+        t_disp = graph_time_ms(lambda: moe.dispatch(ls, d.x, idx, ws), reps)
+        y_perm = moe.expert_ffn(ls, x_perm, offs, d.w_gate, d.w_up, d.w_down, ws)
+        t_ffn = graph_time_ms(lambda: moe.expert_ffn(ls, x_perm, offs, d.w_gate, d.w_up,
+                                                     d.w_down, ws, y_perm=y_perm), reps)
+        out_c = torch.empty_like(out)
+        t_comb = graph_time_ms(lambda: moe.combine(ls, d.x, y_perm, idx, gate, slot_row,
+                                                   out=out_c), reps)
+        t_graph = graph_time_ms(step, reps)
+        es = d.x.element_size()
+        Tk = sh.T * sh.top_k
+        b_route = sh.T * sh.d * es + sh.E * sh.d * 4 + sh.E * 4 + Tk * 8
+        b_disp = 2 * Tk * 4 + Tk * 4 * 2 + 2 * R * sh.d * es
+        b_ffn = U * 3 * sh.ffn * sh.d * es
+        n_zero_tok = int(((idx >= sh.n_routed).any(dim=1)).sum())
+        b_comb = R * sh.d * es + n_zero_tok * sh.d * es + sh.T * sh.d * es + Tk * 12
+        flops_ffn = 6.0 * R * sh.d * sh.ffn
+        comp = {
+            "router_topk": {"ms": t_route, "gbs": b_route / t_route / 1e6},
+            "dispatch": {"ms": t_disp, "gbs": b_disp / t_disp / 1e6},
+            "expert_ffn": {"ms": t_ffn, "gbs": b_ffn / t_ffn / 1e6,
+                           "tflops": flops_ffn / t_ffn / 1e9,
+                           "tensor_frac_of_measured_bf16": flops_ffn / t_ffn / 1e9
+                           / pk["bf16_tflops"]},
+            "combine": {"ms": t_comb, "gbs": b_comb / t_comb / 1e6},
+            "layer_graph": {"ms": t_graph, "tokens_per_s": sh.T / (t_graph / 1e3)},
+            "R": R, "U": U,
+        }
+        ach = b_ffn / t_ffn / 1e6
+        roof = {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": ach / pk["hbm_gbs"], "traffic": None,
+                "kernel": "moe_expert_ffn: grouped_gemm_tc gate/up + down (+ plan)",
+                "algorithmic_bytes": b_ffn,
+                "peak_source": pk["source"] + " hbm_gbs (burst copy)"}
+        if args.traffic_bytes:
+            roof["traffic"] = args.traffic_bytes
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": sh.act_dtype, "data": "synthetic",
+            "config": {"workload": workload_name(sh), "seed": args.seed,
+                       "l2": "inputs larger than L2: the touched expert weights "
+                             f"({U} experts, {U * 3 * sh.ffn * sh.d * 2 / 1e9:.2f} GB) "
+                             "stream from HBM every step",
+                       "parallelism": f"replicas{world}"},
+            "e2e": {"value": world * sh.T / (e2e_ms / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": act_b, "d2h_bytes_per_step": act_b},
+            "gpu_launches": args.steps * moe.launch_count(ls),
+            "roofline": roof,
+            "components": comp,
+            "clocks": clocks,
+        }
+        if not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(sh, inp)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--config", default="decode")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--ref-tokens", type=int, default=8)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--traffic-bytes", type=float, default=None,
+                    help="ncu dram bytes per launch of the dominant kernel pair")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    sh = get_config(args.config)
+    if args.impl == "reference":
+        run_reference(args, sh)
+    else:
+        run_gpu(args, sh)
+
+
+if __name__ == "__main__":
+    main()

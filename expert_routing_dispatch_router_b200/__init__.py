@@ -1,0 +1,274 @@
+"""B200 (sm_100a) library for the forward pass of a mixture-of-experts FFN
+layer with zero-computation (identity) experts: Python binding.
+
+Every step of the layer runs in the CUDA library ``_lib/libmoe.so`` behind the
+C ABI declared in ``include/moe_api.h``. This module only marshals torch CUDA
+tensors into that ABI (pointers, sizes, the current stream); it computes
+nothing itself and has no fallback: if the library is missing, importing the
+binding's functions raises.
+
+Build the library with ``python -m expert_routing_dispatch_router_b200.build``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+from . import build as _build
+
+LIB_PATH = _build.LIB
+HEADER = os.path.join(_build.ROOT, "include", "moe_api.h")
+
+MOE_F32, MOE_BF16 = 0, 1
+STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
+          3: "MOE_ERR_WORKSPACE", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_CHECK"}
+
+
+class MoEError(RuntimeError):
+    def __init__(self, fn: str, status: int, msg: str):
+        super().__init__(f"{fn}: {STATUS.get(status, status)} ({msg})")
+        self.status = status
+
+
+class MoEConfig(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("d", ctypes.c_int32),
+                ("n_routed", ctypes.c_int32), ("n_zero", ctypes.c_int32),
+                ("top_k", ctypes.c_int32), ("ffn", ctypes.c_int32),
+                ("act_dtype", ctypes.c_int32), ("routed_scale", ctypes.c_float)]
+
+
+@dataclass(frozen=True)
+class LayerShape:
+    """Sizes of one layer call (mirrors moe_config_t)."""
+    T: int
+    d: int
+    n_routed: int
+    n_zero: int
+    top_k: int
+    ffn: int
+    act_dtype: torch.dtype = torch.bfloat16
+    routed_scale: float = 1.0
+
+    @property
+    def E(self) -> int:
+        return self.n_routed + self.n_zero
+
+    def c(self) -> MoEConfig:
+        code = {torch.float32: MOE_F32, torch.bfloat16: MOE_BF16}[self.act_dtype]
+        return MoEConfig(self.T, self.d, self.n_routed, self.n_zero, self.top_k,
+                         self.ffn, code, float(self.routed_scale))
+
+
+_lib = None
+P = ctypes.c_void_p
+
+
+def declared_functions():
+    """Names of the functions ``include/moe_api.h`` declares."""
+    with open(HEADER) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"^\s*(?:[\w]+\s*\*?\s+)+\*?(moe_\w+)\(", text, re.M)))
+
+
+def lib():
+    """The loaded CUDA library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(
+                f"CUDA library {LIB_PATH} is missing; build it with "
+                "`python -m expert_routing_dispatch_router_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        C = ctypes.POINTER(MoEConfig)
+        i32 = ctypes.c_int
+        sz = ctypes.c_size_t
+        sig = {
+            "moe_workspace_size": ([C], sz),
+            "moe_route": ([C, P, P, P, P, P, P, P, P, sz, P], i32),
+            "moe_dispatch": ([C, P, P, P, P, P, P, P, P, sz, P], i32),
+            "moe_expert_ffn": ([C, P, P, P, P, P, P, P, sz, P], i32),
+            "moe_combine": ([C, P, P, P, P, P, P, P], i32),
+            "moe_layer_forward": ([C, P, P, P, P, P, P, P, P, P, sz, P], i32),
+            "moe_layer_forward_host": ([C, P, P, P, P, P, P, P, P, P, sz, P], i32),
+            "moe_read_device_error": ([P, P, P], i32),
+            "moe_layer_launch_count": ([C], ctypes.c_int32),
+            "moe_status_string": ([i32], ctypes.c_char_p),
+        }
+        for name, (args, res) in sig.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = L
+    return _lib
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        raise MoEError(fn, status, lib().moe_status_string(status).decode())
+
+
+def _need(t: torch.Tensor, name: str, dtype, shape=None):
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def workspace_size(shape: LayerShape) -> int:
+    return int(lib().moe_workspace_size(ctypes.byref(shape.c())))
+
+
+def alloc_workspace(shape: LayerShape, device="cuda") -> torch.Tensor:
+    """Zeroed workspace (the error word must start at zero)."""
+    n = workspace_size(shape)
+    if n == 0:
+        raise ValueError(f"invalid or unsupported shape {shape}")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def launch_count(shape: LayerShape) -> int:
+    return int(lib().moe_layer_launch_count(ctypes.byref(shape.c())))
+
+
+def route(shape: LayerShape, x, w_router, bias, ws, logits=None, flags=None,
+          stream=None):
+    """Router + top-k + gates -> (topk_idx [T,k] int32, topk_gate [T,k] f32)."""
+    T, E, k = shape.T, shape.E, shape.top_k
+    _need(x, "x", shape.act_dtype, (T, shape.d))
+    _need(w_router, "w_router", torch.float32, (E, shape.d))
+    _need(bias, "bias", torch.float32, (E,))
+    idx = torch.empty(T, k, dtype=torch.int32, device=x.device)
+    gate = torch.empty(T, k, dtype=torch.float32, device=x.device)
+    if logits is not None:
+        _need(logits, "logits", torch.float32, (T, E))
+    if flags is not None:
+        _need(flags, "flags", torch.uint8, (T,))
+    st = lib().moe_route(ctypes.byref(shape.c()), _ptr(x), _ptr(w_router), _ptr(bias),
+                         _ptr(logits), _ptr(idx), _ptr(gate), _ptr(flags), _ptr(ws),
+                         ws.numel(), _stream(stream))
+    _check("moe_route", st)
+    return idx, gate
+
+
+def dispatch(shape: LayerShape, x, topk_idx, ws, stream=None):
+    """-> (counts [E], offsets [N+1], row_token [T*k], slot_row [T*k], x_perm [T*k, d])."""
+    T, k = shape.T, shape.top_k
+    _need(x, "x", shape.act_dtype, (T, shape.d))
+    _need(topk_idx, "topk_idx", torch.int32, (T, k))
+    dev = x.device
+    counts = torch.empty(shape.E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(shape.n_routed + 1, dtype=torch.int32, device=dev)
+    row_token = torch.empty(T * k, dtype=torch.int32, device=dev)
+    slot_row = torch.empty(T * k, dtype=torch.int32, device=dev)
+    x_perm = torch.empty(T * k, shape.d, dtype=shape.act_dtype, device=dev)
+    st = lib().moe_dispatch(ctypes.byref(shape.c()), _ptr(x), _ptr(topk_idx),
+                            _ptr(counts), _ptr(offsets), _ptr(row_token),
+                            _ptr(slot_row), _ptr(x_perm), _ptr(ws), ws.numel(),
+                            _stream(stream))
+    _check("moe_dispatch", st)
+    return counts, offsets, row_token, slot_row, x_perm
+
+
+def expert_ffn(shape: LayerShape, x_perm, offsets, w_gate, w_up, w_down, ws,
+               y_perm=None, stream=None):
+    """-> y_perm [T*k, d] (rows >= R untouched)."""
+    T, k, d, F, N = shape.T, shape.top_k, shape.d, shape.ffn, shape.n_routed
+    _need(x_perm, "x_perm", shape.act_dtype, (T * k, d))
+    _need(offsets, "offsets", torch.int32, (N + 1,))
+    for name, w, shp in (("w_gate", w_gate, (N, F, d)), ("w_up", w_up, (N, F, d)),
+                         ("w_down", w_down, (N, d, F))):
+        _need(w, name, shape.act_dtype, shp)
+    if y_perm is None:
+        y_perm = torch.empty(T * k, d, dtype=shape.act_dtype, device=x_perm.device)
+    _need(y_perm, "y_perm", shape.act_dtype, (T * k, d))
+    st = lib().moe_expert_ffn(ctypes.byref(shape.c()), _ptr(x_perm), _ptr(offsets),
+                              _ptr(w_gate), _ptr(w_up), _ptr(w_down), _ptr(y_perm),
+                              _ptr(ws), ws.numel(), _stream(stream))
+    _check("moe_expert_ffn", st)
+    return y_perm
+
+
+def combine(shape: LayerShape, x, y_perm, topk_idx, topk_gate, slot_row, out=None,
+            stream=None):
+    T, k, d = shape.T, shape.top_k, shape.d
+    _need(x, "x", shape.act_dtype, (T, d))
+    _need(y_perm, "y_perm", shape.act_dtype, (T * k, d))
+    _need(topk_idx, "topk_idx", torch.int32, (T, k))
+    _need(topk_gate, "topk_gate", torch.float32, (T, k))
+    _need(slot_row, "slot_row", torch.int32, (T * k,))
+    if out is None:
+        out = torch.empty(T, d, dtype=shape.act_dtype, device=x.device)
+    _need(out, "out", shape.act_dtype, (T, d))
+    st = lib().moe_combine(ctypes.byref(shape.c()), _ptr(x), _ptr(y_perm),
+                           _ptr(topk_idx), _ptr(topk_gate), _ptr(slot_row), _ptr(out),
+                           _stream(stream))
+    _check("moe_combine", st)
+    return out
+
+
+def layer_forward(shape: LayerShape, x, w_router, bias, w_gate, w_up, w_down, ws,
+                  out=None, counts=None, stream=None):
+    """The whole layer -> out [T, d]; counts [E] (optional) gets slots per expert."""
+    T, d, F, N, E = shape.T, shape.d, shape.ffn, shape.n_routed, shape.E
+    _need(x, "x", shape.act_dtype, (T, d))
+    _need(w_router, "w_router", torch.float32, (E, d))
+    _need(bias, "bias", torch.float32, (E,))
+    if N > 0:
+        for name, w, shp in (("w_gate", w_gate, (N, F, d)), ("w_up", w_up, (N, F, d)),
+                             ("w_down", w_down, (N, d, F))):
+            _need(w, name, shape.act_dtype, shp)
+    if out is None:
+        out = torch.empty(T, d, dtype=shape.act_dtype, device=x.device)
+    _need(out, "out", shape.act_dtype, (T, d))
+    if counts is not None:
+        _need(counts, "counts", torch.int32, (E,))
+    st = lib().moe_layer_forward(ctypes.byref(shape.c()), _ptr(x), _ptr(w_router),
+                                 _ptr(bias), _ptr(w_gate), _ptr(w_up), _ptr(w_down),
+                                 _ptr(out), _ptr(counts), _ptr(ws), ws.numel(),
+                                 _stream(stream))
+    _check("moe_layer_forward", st)
+    return out
+
+
+def layer_forward_host(shape: LayerShape, x_host, w_router, bias, w_gate, w_up,
+                       w_down, ws, out_host, counts_host=None, stream=None):
+    """The whole layer with x and out in (pinned) host memory; asynchronous:
+    synchronise the stream before reading out_host."""
+    T, d, E = shape.T, shape.d, shape.E
+    _need(x_host, "x_host", shape.act_dtype, (T, d))
+    _need(out_host, "out_host", shape.act_dtype, (T, d))
+    if x_host.is_cuda or out_host.is_cuda:
+        raise ValueError("x_host and out_host must be host tensors")
+    if counts_host is not None:
+        _need(counts_host, "counts_host", torch.int32, (E,))
+    st = lib().moe_layer_forward_host(ctypes.byref(shape.c()), _ptr(x_host),
+                                      _ptr(w_router), _ptr(bias), _ptr(w_gate),
+                                      _ptr(w_up), _ptr(w_down), _ptr(out_host),
+                                      _ptr(counts_host), _ptr(ws), ws.numel(),
+                                      _stream(stream))
+    _check("moe_layer_forward_host", st)
+    return out_host
+
+
+def read_device_error(ws, stream=None) -> int:
+    """Waits for the stream; returns (and clears) the workspace error word."""
+    code = ctypes.c_int32(0)
+    lib().moe_read_device_error(_ptr(ws), ctypes.byref(code), _stream(stream))
+    return int(code.value)

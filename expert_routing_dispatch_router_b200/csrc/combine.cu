@@ -1,0 +1,130 @@
+// Combine: gate-weighted sum of each token's expert outputs, with the identity
+// contribution of zero experts.
+//
+// Ascend LongCat-2.0 deployment article (10100.com), "底层定制算子深度优化":
+// a Combine operator that supports zero-computation experts. LongCat-2.0 model
+// card (archdb), "Routed scaling factor": a multiplier on the combined
+// routed-expert output; the library applies it to the routed part only and
+// leaves the identity part of zero experts unscaled.
+//
+//   out[t] = s * sum_{j: idx<N} gate[t,j] * y_perm[slot_row[t,j]]
+//              + sum_{j: idx>=N} gate[t,j] * x[t]
+//
+// Both sums run in fp32 in slot order j = 0..k-1 and the result is rounded
+// once, so the output does not depend on thread timing. Grid: one block row
+// per token, 16-byte vectors along d.
+#include "moe_internal.cuh"
+
+namespace moe {
+namespace {
+
+template <typename AT>
+struct Vec;
+template <>
+struct Vec<__nv_bfloat16> {
+  static constexpr int n = 8;
+  __device__ static void load(const __nv_bfloat16* p, float* v) {
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[2 * i] = __uint_as_float(w[i] << 16);
+      v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+  }
+  __device__ static void store(__nv_bfloat16* p, const float* v) {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const __nv_bfloat162 b = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+      w[i] = *reinterpret_cast<const uint32_t*>(&b);
+    }
+    *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+};
+template <>
+struct Vec<float> {
+  static constexpr int n = 4;
+  __device__ static void load(const float* p, float* v) {
+    const float4 u = *reinterpret_cast<const float4*>(p);
+    v[0] = u.x;
+    v[1] = u.y;
+    v[2] = u.z;
+    v[3] = u.w;
+  }
+  __device__ static void store(float* p, const float* v) {
+    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+  }
+};
+
+template <typename AT>
+__global__ void __launch_bounds__(128)
+    combine_kernel(const AT* __restrict__ x, const AT* __restrict__ y,
+                   const int32_t* __restrict__ idx,
+                   const float* __restrict__ gate,
+                   const int32_t* __restrict__ slot_row, AT* __restrict__ out,
+                   int64_t d, int N, int k, float s) {
+  constexpr int V = Vec<AT>::n;
+  __shared__ int32_t s_row[kMaxTopK];
+  __shared__ float s_gate[kMaxTopK];
+  __shared__ int32_t s_zero[kMaxTopK];
+  const int64_t t = blockIdx.x;
+  if (threadIdx.x < k) {
+    const int e = idx[t * k + threadIdx.x];
+    s_row[threadIdx.x] = slot_row[t * k + threadIdx.x];
+    s_gate[threadIdx.x] = gate[t * k + threadIdx.x];
+    s_zero[threadIdx.x] = (e >= N) ? 1 : 0;
+  }
+  __syncthreads();
+  const int64_t col = ((int64_t)blockIdx.y * blockDim.x + threadIdx.x) * V;
+  if (col >= d) return;
+  float racc[V], zacc[V], v[V];
+#pragma unroll
+  for (int i = 0; i < V; ++i) racc[i] = zacc[i] = 0.f;
+  bool have_x = false;
+  float xv[V];
+  for (int j = 0; j < k; ++j) {
+    const float g = s_gate[j];
+    if (s_zero[j]) {
+      if (!have_x) {
+        Vec<AT>::load(x + t * d + col, xv);
+        have_x = true;
+      }
+#pragma unroll
+      for (int i = 0; i < V; ++i) zacc[i] = fmaf(g, xv[i], zacc[i]);
+    } else {
+      const int64_t r = s_row[j];
+      if (r < 0) continue;
+      Vec<AT>::load(y + r * d + col, v);
+#pragma unroll
+      for (int i = 0; i < V; ++i) racc[i] = fmaf(g, v[i], racc[i]);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < V; ++i) v[i] = fmaf(s, racc[i], zacc[i]);
+  Vec<AT>::store(out + t * d + col, v);
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const Shape& sh, const void* x, const void* y_perm,
+                           const int32_t* idx, const float* gate,
+                           const int32_t* slot_row, void* out, cudaStream_t st) {
+  const int V = sh.bf16 ? 8 : 4;
+  const int64_t vecs = sh.d / V;
+  const int threads = 128;
+  dim3 grid((unsigned)sh.T, (unsigned)((vecs + threads - 1) / threads));
+  if (sh.bf16)
+    combine_kernel<__nv_bfloat16><<<grid, threads, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(x),
+        static_cast<const __nv_bfloat16*>(y_perm), idx, gate, slot_row,
+        static_cast<__nv_bfloat16*>(out), sh.d, (int)sh.N, (int)sh.k, sh.s);
+  else
+    combine_kernel<float><<<grid, threads, 0, st>>>(
+        static_cast<const float*>(x), static_cast<const float*>(y_perm), idx,
+        gate, slot_row, static_cast<float*>(out), sh.d, (int)sh.N, (int)sh.k,
+        sh.s);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

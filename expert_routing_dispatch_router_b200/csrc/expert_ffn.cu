@@ -1,0 +1,554 @@
+// Routed experts over the dispatched rows: a grouped SwiGLU FFN,
+//   h = silu(x W_gate[e]^T) * (x W_up[e]^T),   y = h W_down[e]^T,
+// for every expert e over its contiguous segment of rows [offsets[e],
+// offsets[e+1]). LongCat-2.0 model card (archdb), "Mixture of experts" (expert
+// dim) and "Feed-forward" (activation not disclosed; SwiGLU is the reading).
+//
+// Tensor-core path (bf16, d and F multiples of 128): one persistent kernel per
+// GEMM (gate/up, then down), warp-specialised for sm_100a:
+//   warp 0      TMA producer: weight tiles and token tiles -> smem ring
+//   warp 1      MMA issuer: tcgen05.mma into TMEM (fp32), tcgen05.commit
+//   warps 2..5  epilogue: tcgen05.ld from TMEM, SwiGLU, bf16 stores
+// The operands are swapped relative to the usual token-major GEMM: 128 rows
+// of an expert's weight matrix fill the MMA's M = 128 and the expert's tokens
+// (up to 128 per tile, rounded up to a multiple of 16) are its N. A decode
+// batch gives an expert ~3 tokens, so this keeps the tensor work at N = 16
+// instead of padding tokens to M = 128, and the kernel streams weights at
+// HBM speed. The gate/up kernel loads the W_gate and W_up tiles of the same
+// 128 rows and issues two MMAs against one token tile, so the epilogue has
+// both accumulators of a row at hand. TMEM holds two accumulator buffers so
+// the epilogue of one tile overlaps the MMAs of the next.
+//
+// Work unit = (expert, 128-row weight tile m, token tile). Units are numbered
+// expert-major, then m, then token tile, so CTAs that run at the same time
+// share weight tiles through L2. A tiny plan kernel turns offsets[] into
+// per-expert token-tile prefix sums on the device; no host sync is needed.
+//
+// Every mbarrier wait is bounded (about 2 s); on expiry the kernel records an
+// error code in the workspace, the other roles stop, outstanding TMA loads and
+// MMAs are waited for (again bounded), TMEM is freed and the kernel returns.
+//
+// CUDA-core path (f32, or shapes the tensor-core path does not take): one warp
+// per output element, fp32 accumulation, same rounding points (h is stored in
+// the activation type).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "moe_internal.cuh"
+#include "sm100_ptx.cuh"
+
+namespace moe {
+namespace {
+
+// ------------------------------------------------------------------ plan --
+// tile_start[e] = sum over routed e' < e of ceil(count[e'] / kTileTokens);
+// tile_start[N] = total token tiles. One block; N <= 1024.
+__global__ void __launch_bounds__(1024)
+    gemm_plan_kernel(const int32_t* __restrict__ offsets, int N,
+                     int32_t* __restrict__ tile_start) {
+  __shared__ int32_t warp_sums[32];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  int32_t v = 0;
+  if ((int)threadIdx.x < N) {
+    const int32_t n = offsets[threadIdx.x + 1] - offsets[threadIdx.x];
+    v = (n + kTileTokens - 1) / kTileTokens;
+  }
+  int32_t incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int32_t o = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += o;
+  }
+  if (lane == 31) warp_sums[wid] = incl;
+  __syncthreads();
+  if (wid == 0) {
+    int32_t s = warp_sums[lane];
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int32_t o = __shfl_up_sync(0xffffffffu, s, off);
+      if (lane >= off) s += o;
+    }
+    warp_sums[lane] = s;
+  }
+  __syncthreads();
+  const int32_t before = (wid > 0 ? warp_sums[wid - 1] : 0) + incl - v;
+  if ((int)threadIdx.x < N) tile_start[threadIdx.x] = before;
+  if (threadIdx.x == 0) tile_start[N] = warp_sums[31];
+}
+
+// ------------------------------------------------------- tensor-core path --
+constexpr int BM = 128;  // weight rows per tile (MMA M)
+constexpr int BK = 64;   // contraction elements per stage: 128-byte rows
+constexpr int BN = kTileTokens;  // token rows per tile (MMA N, max)
+constexpr int kThreads = 192;
+constexpr uint32_t kTileBytes = BM * BK * 2;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kAccStride = 256;  // TMEM columns per accumulator buffer
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+template <bool GATEUP>
+struct Cfg {
+  static constexpr int kNumA = GATEUP ? 2 : 1;
+  static constexpr int kStages = GATEUP ? 4 : 6;
+  static constexpr uint32_t kStageBytes = (kNumA + 1) * kTileBytes;
+  static constexpr uint32_t kBarOff = kStages * kStageBytes;
+  static constexpr uint32_t kTabOff = kBarOff + 256;
+  static constexpr uint32_t kSmemBytes =
+      1024 + kTabOff + 2 * 4 * (kMaxExperts + 1);
+};
+
+struct GemmArgs {
+  const int32_t* offsets;     // [N+1] row offsets per expert
+  const int32_t* tile_start;  // [N+1] token-tile prefix per expert
+  __nv_bfloat16* out;         // [rows_cap, out_cols]
+  int32_t* err;               // workspace error word
+  int N;
+  int num_kb;    // contraction length / BK
+  int out_cols;  // F for gate/up, d for down
+  int m_tiles;   // out_cols / BM
+};
+
+struct Unit {
+  int e, m, row0, n_valid, n_mma;
+};
+
+__device__ __forceinline__ Unit decode_unit(int u, const int* s_tiles,
+                                            const int* s_offs, int N,
+                                            int m_tiles) {
+  int lo = 0, hi = N - 1;  // largest e with m_tiles * tile_start[e] <= u
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (m_tiles * s_tiles[mid] <= u)
+      lo = mid;
+    else
+      hi = mid - 1;
+  }
+  Unit un;
+  un.e = lo;
+  const int ntiles = s_tiles[lo + 1] - s_tiles[lo];
+  const int local = u - m_tiles * s_tiles[lo];
+  un.m = local / ntiles;
+  const int tt = local - un.m * ntiles;
+  un.row0 = s_offs[lo] + tt * BN;
+  const int rem = s_offs[lo + 1] - un.row0;
+  un.n_valid = rem < BN ? rem : BN;
+  un.n_mma = (un.n_valid + 15) & ~15;
+  return un;
+}
+
+// Bounded wait on an mbarrier phase. Returns false when the CTA was told to
+// stop or when the limit ran out (then it tells the CTA to stop and records
+// the error).
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity,
+                                             volatile int* abort_flag,
+                                             int32_t* err) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = ptx::global_timer_ns();
+  while (true) {
+    for (int i = 0; i < 64; ++i)
+      if (ptx::mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (ptx::global_timer_ns() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      atomicCAS(err, 0, kErrWaitTimeout);
+      return false;
+    }
+  }
+}
+
+// Bounded wait that ignores the stop flag (used while cleaning up).
+__device__ __forceinline__ void wait_cleanup(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = ptx::global_timer_ns();
+  while (!ptx::mbar_try_wait(bar, parity))
+    if (ptx::global_timer_ns() - t0 > kWaitLimitNs) return;
+}
+
+__device__ __forceinline__ float silu_f(float z) { return z / (1.0f + __expf(-z)); }
+
+template <bool GATEUP>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0,
+                           const __grid_constant__ CUtensorMap tmA1,
+                           const __grid_constant__ CUtensorMap tmB16,
+                           const __grid_constant__ CUtensorMap tmB128,
+                           const GemmArgs args) {
+  using C = Cfg<GATEUP>;
+  constexpr int S = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = ptx::smem_addr(smem);
+  const uint32_t bars = sbase + C::kBarOff;
+  auto full_bar = [&](int s) { return bars + 8u * s; };
+  auto empty_bar = [&](int s) { return bars + 8u * (S + s); };
+  auto tfull_bar = [&](int b) { return bars + 8u * (2 * S + b); };
+  auto tempty_bar = [&](int b) { return bars + 8u * (2 * S + 2 + b); };
+  const uint32_t mma_done_bar = bars + 8u * (2 * S + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + 8 * (2 * S + 5));
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* s_tiles = reinterpret_cast<int*>(smem + C::kTabOff);
+  int* s_offs = s_tiles + (kMaxExperts + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int N = args.N;
+  for (int i = threadIdx.x; i <= N; i += blockDim.x) {
+    s_tiles[i] = args.tile_start[i];
+    s_offs[i] = args.offsets[i];
+  }
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      ptx::mbar_init(full_bar(s), 1);
+      ptx::mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(tfull_bar(b), 1);
+      ptx::mbar_init(tempty_bar(b), 4);
+    }
+    ptx::mbar_init(mma_done_bar, 1);
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    ptx::prefetch_tensormap(&tmA0);
+    if (GATEUP) ptx::prefetch_tensormap(&tmA1);
+    ptx::prefetch_tensormap(&tmB16);
+    ptx::prefetch_tensormap(&tmB128);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(ptx::smem_addr(tmem_slot), kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
+  const int total_units = s_tiles[N] * args.m_tiles;
+
+  if (warp == 0) {
+    // ---------------------------------------------------- TMA producer --
+    if (lane == 0) {
+      const uint64_t pol_w = ptx::policy_evict_first();
+      const uint64_t pol_x = ptx::policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0, armed = 0, armed_par = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
+        const Unit un = decode_unit(u, s_tiles, s_offs, N, args.m_tiles);
+        const int arow = un.e * args.out_cols + un.m * BM;
+        const uint32_t bytes = C::kNumA * kTileBytes + (uint32_t)un.n_mma * 128u;
+        for (int kb = 0; kb < args.num_kb; ++kb) {
+          if (!wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, args.err)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = full_bar(stage);
+          ptx::mbar_arrive_expect_tx(fb, bytes);
+          const uint32_t a0 = sbase + stage * C::kStageBytes;
+          ptx::tma_load_2d(&tmA0, a0, fb, kb * BK, arow, pol_w);
+          if (GATEUP) ptx::tma_load_2d(&tmA1, a0 + kTileBytes, fb, kb * BK, arow, pol_w);
+          const uint32_t b0 = a0 + C::kNumA * kTileBytes;
+          if (un.n_mma == BN) {
+            ptx::tma_load_2d(&tmB128, b0, fb, kb * BK, un.row0, pol_x);
+          } else {
+            for (int j = 0; j < un.n_mma / 16; ++j)
+              ptx::tma_load_2d(&tmB16, b0 + j * 2048u, fb, kb * BK, un.row0 + 16 * j,
+                               pol_x);
+          }
+          armed |= 1u << stage;
+          armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {  // let our own loads land before the CTA goes away
+        for (int s = 0; s < S; ++s)
+          if ((armed >> s) & 1u) wait_cleanup(full_bar(s), (armed_par >> s) & 1u);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------ MMA issuer --
+    if (lane == 0) {
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true, issued = false;
+      for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
+        const Unit un = decode_unit(u, s_tiles, s_offs, N, args.m_tiles);
+        if (!wait_bounded(tempty_bar(acc), acc_phase ^ 1u, abort_flag, args.err)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t idesc = ptx::idesc_bf16_f32(BM, un.n_mma);
+        const uint32_t d0 = tmem_base + (uint32_t)acc * kAccStride;
+        for (int kb = 0; kb < args.num_kb; ++kb) {
+          if (!wait_bounded(full_bar(stage), phase, abort_flag, args.err)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t a0 = sbase + stage * C::kStageBytes;
+          const uint32_t b0 = a0 + C::kNumA * kTileBytes;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t bdesc = ptx::desc_k_sw128(b0 + kk * 32);
+            const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
+            ptx::mma_bf16(d0, ptx::desc_k_sw128(a0 + kk * 32), bdesc, idesc, accum);
+            if (GATEUP)
+              ptx::mma_bf16(d0 + 128, ptx::desc_k_sw128(a0 + kTileBytes + kk * 32),
+                            bdesc, idesc, accum);
+          }
+          issued = true;
+          ptx::mma_commit(empty_bar(stage));
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        ptx::mma_commit(tfull_bar(acc));
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      if (!ok && issued) {  // the MMAs already issued must finish before TMEM is freed
+        ptx::mma_commit(mma_done_bar);
+        wait_cleanup(mma_done_bar, 0);
+      }
+    }
+  } else {
+    // -------------------------------------------------------- epilogue --
+    const int ew = warp & 3;  // TMEM lane quarter this warp may access
+    const int lrow = ew * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int u = blockIdx.x; u < total_units; u += gridDim.x) {
+      const Unit un = decode_unit(u, s_tiles, s_offs, N, args.m_tiles);
+      const bool ok = wait_bounded(tfull_bar(acc), acc_phase, abort_flag, args.err);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      ptx::tc_fence_after();
+      const uint32_t tb = tmem_base + (static_cast<uint32_t>(ew * 32) << 16) +
+                          (uint32_t)acc * kAccStride;
+      const int64_t col = (int64_t)un.m * BM + lrow;
+      __nv_bfloat16* outp = args.out + (int64_t)un.row0 * args.out_cols + col;
+      for (int c0 = 0; c0 < un.n_mma; c0 += 16) {
+        float g[16], v[16];
+        if (GATEUP)
+          ptx::tmem_ld16x2(tb + c0, tb + 128 + c0, g, v);
+        else
+          ptx::tmem_ld16(tb + c0, g);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          if (c0 + c < un.n_valid) {
+            const float r = GATEUP ? silu_f(g[c]) * v[c] : g[c];
+            outp[(int64_t)(c0 + c) * args.out_cols] = __float2bfloat16_rn(r);
+          }
+        }
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(tempty_bar(acc));
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// Row-major bf16 matrix [rows, cols] seen as a 2-D tensor, box = 64 columns
+// (128 bytes, 128-byte swizzle) x box_rows rows. Rows past `rows` read as 0.
+bool make_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+              uint32_t box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+             strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool GATEUP>
+cudaError_t launch_tc(const CUtensorMap& a0, const CUtensorMap& a1,
+                      const CUtensorMap& b16, const CUtensorMap& b128,
+                      const GemmArgs& args, cudaStream_t st) {
+  using C = Cfg<GATEUP>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_tc_kernel<GATEUP>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  grouped_gemm_tc_kernel<GATEUP><<<num_sms(), kThreads, C::kSmemBytes, st>>>(
+      a0, a1, b16, b128, args);
+  return cudaGetLastError();
+}
+
+// --------------------------------------------------------- CUDA-core path --
+__device__ __forceinline__ int expert_of_row(const int32_t* offsets, int N, int64_t r) {
+  int lo = 0, hi = N - 1;  // largest e with offsets[e] <= r
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (offsets[mid] <= r)
+      lo = mid;
+    else
+      hi = mid - 1;
+  }
+  return lo;
+}
+
+template <typename AT>
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  return v;
+}
+
+// h[r, f] = silu(x_perm[r] . w_gate[e, f]) * (x_perm[r] . w_up[e, f])
+template <typename AT>
+__global__ void __launch_bounds__(256)
+    ffn_gateup_simt_kernel(const AT* __restrict__ x, const int32_t* __restrict__ offsets,
+                           int N, const AT* __restrict__ wg, const AT* __restrict__ wu,
+                           AT* __restrict__ h, int64_t d, int64_t F) {
+  const int64_t R = offsets[N];
+  const int lane = threadIdx.x & 31;
+  const int64_t nw = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t w = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       w < R * F; w += nw) {
+    const int64_t r = w / F, f = w - (w / F) * F;
+    const int e = expert_of_row(offsets, N, r);
+    const AT* xr = x + r * d;
+    const AT* gr = wg + ((int64_t)e * F + f) * d;
+    const AT* ur = wu + ((int64_t)e * F + f) * d;
+    float a = 0.f, u = 0.f;
+    for (int64_t i = lane; i < d; i += 32) {
+      const float xv = to_f32(xr[i]);
+      a = fmaf(to_f32(gr[i]), xv, a);
+      u = fmaf(to_f32(ur[i]), xv, u);
+    }
+    a = warp_sum<AT>(a);
+    u = warp_sum<AT>(u);
+    if (lane == 0) h[r * F + f] = from_f32<AT>(a / (1.0f + expf(-a)) * u);
+  }
+}
+
+// y[r, n] = h[r] . w_down[e, n]
+template <typename AT>
+__global__ void __launch_bounds__(256)
+    ffn_down_simt_kernel(const AT* __restrict__ h, const int32_t* __restrict__ offsets,
+                         int N, const AT* __restrict__ wd, AT* __restrict__ y,
+                         int64_t d, int64_t F) {
+  const int64_t R = offsets[N];
+  const int lane = threadIdx.x & 31;
+  const int64_t nw = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t w = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       w < R * d; w += nw) {
+    const int64_t r = w / d, n = w - (w / d) * d;
+    const int e = expert_of_row(offsets, N, r);
+    const AT* hr = h + r * F;
+    const AT* dr = wd + ((int64_t)e * d + n) * F;
+    float acc = 0.f;
+    for (int64_t f = lane; f < F; f += 32) acc = fmaf(to_f32(dr[f]), to_f32(hr[f]), acc);
+    acc = warp_sum<AT>(acc);
+    if (lane == 0) y[r * d + n] = from_f32<AT>(acc);
+  }
+}
+
+template <typename AT>
+cudaError_t launch_simt(const Shape& sh, const void* x_perm, const int32_t* offsets,
+                        const void* wg, const void* wu, const void* wd, void* h,
+                        void* y, cudaStream_t st) {
+  const unsigned blocks = (unsigned)num_sms() * 16;
+  ffn_gateup_simt_kernel<AT><<<blocks, 256, 0, st>>>(
+      static_cast<const AT*>(x_perm), offsets, (int)sh.N, static_cast<const AT*>(wg),
+      static_cast<const AT*>(wu), static_cast<AT*>(h), sh.d, sh.F);
+  ffn_down_simt_kernel<AT><<<blocks, 256, 0, st>>>(
+      static_cast<const AT*>(h), offsets, (int)sh.N, static_cast<const AT*>(wd),
+      static_cast<AT*>(y), sh.d, sh.F);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool expert_ffn_uses_tensor_cores(const Shape& sh) {
+  return sh.bf16 && sh.d % 128 == 0 && sh.F % 128 == 0 && sh.N <= kMaxExperts;
+}
+
+int expert_ffn_launch_count(const Shape& sh) {
+  if (sh.N == 0) return 0;
+  return expert_ffn_uses_tensor_cores(sh) ? 3 : 2;
+}
+
+cudaError_t launch_expert_ffn(const Shape& sh, const void* x_perm,
+                              const int32_t* offsets, const void* w_gate,
+                              const void* w_up, const void* w_down, void* h,
+                              void* y_perm, int32_t* tile_start, int32_t* err,
+                              cudaStream_t st) {
+  if (sh.N == 0 || sh.T == 0) return cudaSuccess;
+  if (!expert_ffn_uses_tensor_cores(sh)) {
+    if (sh.bf16)
+      return launch_simt<__nv_bfloat16>(sh, x_perm, offsets, w_gate, w_up, w_down, h,
+                                        y_perm, st);
+    return launch_simt<float>(sh, x_perm, offsets, w_gate, w_up, w_down, h, y_perm, st);
+  }
+  const uint64_t rows_cap = (uint64_t)(sh.T * sh.k);
+  CUtensorMap wg_map, wu_map, wd_map, x16, x128, h16, h128;
+  const bool ok =
+      make_map(&wg_map, w_gate, (uint64_t)(sh.N * sh.F), (uint64_t)sh.d, BM) &&
+      make_map(&wu_map, w_up, (uint64_t)(sh.N * sh.F), (uint64_t)sh.d, BM) &&
+      make_map(&wd_map, w_down, (uint64_t)(sh.N * sh.d), (uint64_t)sh.F, BM) &&
+      make_map(&x16, x_perm, rows_cap, (uint64_t)sh.d, 16) &&
+      make_map(&x128, x_perm, rows_cap, (uint64_t)sh.d, BN) &&
+      make_map(&h16, h, rows_cap, (uint64_t)sh.F, 16) &&
+      make_map(&h128, h, rows_cap, (uint64_t)sh.F, BN);
+  if (!ok) return cudaErrorInvalidValue;
+
+  gemm_plan_kernel<<<1, 1024, 0, st>>>(offsets, (int)sh.N, tile_start);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+
+  GemmArgs gu;
+  gu.offsets = offsets;
+  gu.tile_start = tile_start;
+  gu.out = static_cast<__nv_bfloat16*>(h);
+  gu.err = err;
+  gu.N = (int)sh.N;
+  gu.num_kb = (int)(sh.d / BK);
+  gu.out_cols = (int)sh.F;
+  gu.m_tiles = (int)(sh.F / BM);
+  e = launch_tc<true>(wg_map, wu_map, x16, x128, gu, st);
+  if (e != cudaSuccess) return e;
+
+  GemmArgs dn = gu;
+  dn.out = static_cast<__nv_bfloat16*>(y_perm);
+  dn.num_kb = (int)(sh.F / BK);
+  dn.out_cols = (int)sh.d;
+  dn.m_tiles = (int)(sh.d / BM);
+  return launch_tc<false>(wd_map, wd_map, h16, h128, dn, st);
+}
+
+}  // namespace moe

@@ -1,0 +1,100 @@
+// Internal declarations shared by the CUDA sources of the MoE library:
+// workspace layout, launcher prototypes and small device helpers.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/moe_api.h"
+
+namespace moe {
+
+constexpr int kMaxExperts = 1024;  // top-k keeps E/32 keys per lane
+constexpr int kMaxTopK = 32;       // one gate per lane
+constexpr int kChunkTokens = 256;  // tokens per dispatch block
+constexpr int kTileTokens = 128;   // token tile of the expert GEMMs
+constexpr int kWsAlign = 1024;
+
+// Device error codes written into the workspace header.
+constexpr int kErrWaitTimeout = 1;
+constexpr int kErrBadExpertId = 2;
+
+// Layout of the workspace (byte offsets from its base). Built on the host
+// from the config alone; every region is kWsAlign-aligned.
+struct WsLayout {
+  size_t header;       // int32[64]: [0] error code, [1] error detail
+  size_t logits;       // float [splits, T, E] router partial sums
+  size_t topk_idx;     // int32 [T, k]
+  size_t topk_gate;    // float [T, k]
+  size_t chunk_base;   // int32 [nchunks, E]
+  size_t counts;       // int32 [E]
+  size_t offsets;      // int32 [N + 1]
+  size_t row_token;    // int32 [T*k]
+  size_t slot_row;     // int32 [T*k]
+  size_t tile_start;   // int32 [N + 1] (expert GEMM plan)
+  size_t x_perm;       // act   [T*k, d]
+  size_t h;            // act   [T*k, F]
+  size_t y_perm;       // act   [T*k, d]
+  size_t x_stage;      // act   [T, d]   (host-buffer entry point)
+  size_t out_stage;    // act   [T, d]
+  size_t total;
+};
+
+struct Shape {
+  int64_t T, d, N, Z, E, k, F;
+  int es;  // bytes per activation element
+  float s;
+  bool bf16;
+  int64_t nchunks;
+};
+
+WsLayout ws_layout(const Shape& sh);
+
+// ---- launchers (each returns cudaGetLastError() after its launches) ----
+int router_splits(const Shape& sh);
+cudaError_t launch_router(const Shape& sh, const void* x, const float* w_r,
+                          const float* bias, float* part, int32_t* idx,
+                          float* gate, uint8_t* flags, float* logits_out,
+                          cudaStream_t st);
+cudaError_t launch_dispatch(const Shape& sh, const void* x, const int32_t* idx,
+                            int32_t* chunk_base, int32_t* counts,
+                            int32_t* offsets, int32_t* row_token,
+                            int32_t* slot_row, void* x_perm, int32_t* err,
+                            cudaStream_t st);
+cudaError_t launch_expert_ffn(const Shape& sh, const void* x_perm,
+                              const int32_t* offsets, const void* w_gate,
+                              const void* w_up, const void* w_down, void* h,
+                              void* y_perm, int32_t* tile_start, int32_t* err,
+                              cudaStream_t st);
+cudaError_t launch_combine(const Shape& sh, const void* x, const void* y_perm,
+                           const int32_t* idx, const float* gate,
+                           const int32_t* slot_row, void* out, cudaStream_t st);
+int expert_ffn_launch_count(const Shape& sh);
+bool expert_ffn_uses_tensor_cores(const Shape& sh);
+int num_sms();
+
+// ---- device helpers ----
+__device__ __forceinline__ float bf16_to_f32(uint16_t b) {
+  return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+
+template <typename T>
+__device__ __forceinline__ float to_f32(T v);
+template <>
+__device__ __forceinline__ float to_f32<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) {
+  return __bfloat162float(v);
+}
+
+template <typename T>
+__device__ __forceinline__ T from_f32(float v);
+template <>
+__device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) {
+  return __float2bfloat16_rn(v);
+}
+
+}  // namespace moe

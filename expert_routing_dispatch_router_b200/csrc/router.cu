@@ -1,0 +1,298 @@
+// Router: fp32-accumulated logits GEMM, correction bias, warp-level top-k and
+// gates.
+//
+// LongCat-2.0 model card (archdb), "Mixture of experts": one router classifier
+// [E, d] scores routed and zero experts together, with a per-expert
+// e_score_correction_bias; 12 experts per token. The score function and the
+// renormalisation are not disclosed there; the library uses the reading that
+// the bias steers selection only and that the gates are the softmax of the
+// selected raw logits (they sum to 1).
+//
+// Kernel 1 (router_logits_kernel): CUDA-core GEMM in fp32. The contraction is
+// split over blockIdx.z so that a decode batch (T ~ 64) still spreads the
+// router weights over many SMs; each split writes its partial sums to the
+// workspace and kernel 2 adds them in a fixed order, so results are
+// bit-reproducible run to run.
+//
+// Kernel 2 (topk_kernel): one warp per token. The E keys sit in registers,
+// ceil(E/32) per lane. k+1 rounds of a warp arg-max (ties to the lower id)
+// give the selection in descending key order and the margin between the k-th
+// and (k+1)-th key.
+#include <float.h>
+#include <math.h>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int RT = 64;   // tokens per CTA
+constexpr int RE = 32;   // experts per CTA
+constexpr int RK = 32;   // contraction chunk
+constexpr int kRouterThreads = 256;
+
+template <typename XT>
+__device__ __forceinline__ void load_x_chunk(const XT* x, int64_t T, int64_t d,
+                                             int64_t t0, int64_t k0,
+                                             int64_t kend,
+                                             float (*xs)[RT + 4]);
+
+// bf16 x: 64 tokens x 32 k = 256 vectors of 8 elements, one per thread.
+template <>
+__device__ __forceinline__ void load_x_chunk<__nv_bfloat16>(
+    const __nv_bfloat16* x, int64_t T, int64_t d, int64_t t0, int64_t k0,
+    int64_t kend, float (*xs)[RT + 4]) {
+  const int tid = threadIdx.x;
+  const int tt = tid >> 2;
+  const int kk = (tid & 3) * 8;
+  const int64_t t = t0 + tt;
+  const int64_t k = k0 + kk;
+  uint4 v = make_uint4(0, 0, 0, 0);
+  if (t < T && k < kend)
+    v = *reinterpret_cast<const uint4*>(x + t * d + k);
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    xs[kk + 2 * i][tt] = __uint_as_float(w[i] << 16);
+    xs[kk + 2 * i + 1][tt] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+
+// f32 x: 64 tokens x 32 k = 512 vectors of 4 elements, two per thread.
+template <>
+__device__ __forceinline__ void load_x_chunk<float>(const float* x, int64_t T,
+                                                    int64_t d, int64_t t0,
+                                                    int64_t k0, int64_t kend,
+                                                    float (*xs)[RT + 4]) {
+#pragma unroll
+  for (int rep = 0; rep < 2; ++rep) {
+    const int v_id = threadIdx.x + rep * kRouterThreads;
+    const int tt = v_id >> 3;
+    const int kk = (v_id & 7) * 4;
+    const int64_t t = t0 + tt;
+    const int64_t k = k0 + kk;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (t < T && k < kend) v = *reinterpret_cast<const float4*>(x + t * d + k);
+    xs[kk + 0][tt] = v.x;
+    xs[kk + 1][tt] = v.y;
+    xs[kk + 2][tt] = v.z;
+    xs[kk + 3][tt] = v.w;
+  }
+}
+
+// part[z][t][e] = sum over this split's k of x[t,k] * w_r[e,k]  (fp32 FFMA)
+template <typename XT>
+__global__ void __launch_bounds__(kRouterThreads)
+    router_logits_kernel(const XT* __restrict__ x, const float* __restrict__ w_r,
+                         float* __restrict__ part, int64_t T, int64_t d,
+                         int64_t E, int64_t k_per_split) {
+  __shared__ __align__(16) float xs[RK][RT + 4];
+  __shared__ __align__(16) float wsm[RK][RE + 4];
+  const int tid = threadIdx.x;
+  const int tx = tid & 15;  // expert pair
+  const int ty = tid >> 4;  // token quad
+  const int64_t e0 = (int64_t)blockIdx.x * RE;
+  const int64_t t0 = (int64_t)blockIdx.y * RT;
+  const int64_t kbeg = (int64_t)blockIdx.z * k_per_split;
+  const int64_t kend = min(d, kbeg + k_per_split);
+
+  float acc[4][2];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = 0.f;
+
+  for (int64_t k0 = kbeg; k0 < kend; k0 += RK) {
+    load_x_chunk<XT>(x, T, d, t0, k0, kend, xs);
+    {  // 32 experts x 32 k floats = 256 float4, one per thread
+      const int ee = tid >> 3;
+      const int kk = (tid & 7) * 4;
+      const int64_t e = e0 + ee;
+      const int64_t k = k0 + kk;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (e < E && k < kend)
+        v = *reinterpret_cast<const float4*>(w_r + e * d + k);
+      wsm[kk + 0][ee] = v.x;
+      wsm[kk + 1][ee] = v.y;
+      wsm[kk + 2][ee] = v.z;
+      wsm[kk + 3][ee] = v.w;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int kk = 0; kk < RK; ++kk) {
+      const float4 xv = *reinterpret_cast<const float4*>(&xs[kk][ty * 4]);
+      const float2 wv = *reinterpret_cast<const float2*>(&wsm[kk][tx * 2]);
+      acc[0][0] = fmaf(xv.x, wv.x, acc[0][0]);
+      acc[0][1] = fmaf(xv.x, wv.y, acc[0][1]);
+      acc[1][0] = fmaf(xv.y, wv.x, acc[1][0]);
+      acc[1][1] = fmaf(xv.y, wv.y, acc[1][1]);
+      acc[2][0] = fmaf(xv.z, wv.x, acc[2][0]);
+      acc[2][1] = fmaf(xv.z, wv.y, acc[2][1]);
+      acc[3][0] = fmaf(xv.w, wv.x, acc[3][0]);
+      acc[3][1] = fmaf(xv.w, wv.y, acc[3][1]);
+    }
+    __syncthreads();
+  }
+  float* out = part + (int64_t)blockIdx.z * T * E;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t t = t0 + ty * 4 + i;
+    if (t >= T) continue;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int64_t e = e0 + tx * 2 + j;
+      if (e < E) out[t * E + e] = acc[i][j];
+    }
+  }
+}
+
+struct Cand {
+  float key;
+  float logit;
+  int e;
+};
+
+// a beats b: larger key, ties to the lower expert id
+__device__ __forceinline__ bool beats(float ka, int ea, float kb, int eb) {
+  return ka > kb || (ka == kb && ea < eb);
+}
+
+template <int PL>
+__global__ void __launch_bounds__(256)
+    topk_kernel(const float* __restrict__ part, int nsplit,
+                const float* __restrict__ bias, float* __restrict__ logits_out,
+                int32_t* __restrict__ idx_out, float* __restrict__ gate_out,
+                uint8_t* __restrict__ flags, int64_t T, int E, int k) {
+  const int lane = threadIdx.x & 31;
+  const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T) return;
+
+  float lg[PL], key[PL];
+#pragma unroll
+  for (int i = 0; i < PL; ++i) {
+    const int e = lane + 32 * i;
+    lg[i] = 0.f;
+    key[i] = -INFINITY;
+    if (e < E) {
+      float l = 0.f;
+      for (int z = 0; z < nsplit; ++z) l += part[((int64_t)z * T + t) * E + e];
+      lg[i] = l;
+      float kv = l + bias[e];
+      key[i] = (kv != kv) ? -INFINITY : kv;  // a NaN key never wins
+      if (logits_out) logits_out[t * E + e] = l;
+    }
+  }
+
+  uint32_t taken = 0;  // bit i: expert lane + 32 i already selected
+  float kth_key = 0.f, next_key = -INFINITY;
+  float my_logit = 0.f;
+  int my_e = 0;
+  const int rounds = (k < E) ? k + 1 : k;
+  for (int j = 0; j < rounds; ++j) {
+    float bk = -INFINITY, bl = 0.f;
+    int be = 0x7fffffff;
+#pragma unroll
+    for (int i = 0; i < PL; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E && !((taken >> i) & 1u) && beats(key[i], e, bk, be)) {
+        bk = key[i];
+        be = e;
+        bl = lg[i];
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float ok = __shfl_xor_sync(0xffffffffu, bk, off);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+      const float ol = __shfl_xor_sync(0xffffffffu, bl, off);
+      if (beats(ok, oe, bk, be)) {
+        bk = ok;
+        be = oe;
+        bl = ol;
+      }
+    }
+    if (j < k) {
+      if (lane == (be & 31)) taken |= 1u << (be >> 5);
+      if (lane == j) {
+        my_logit = bl;
+        my_e = be;
+      }
+      kth_key = bk;
+    } else {
+      next_key = bk;
+    }
+  }
+
+  // gates: softmax of the selected raw logits
+  float m = (lane < k) ? my_logit : -INFINITY;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1)
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  float p = (lane < k) ? expf(my_logit - m) : 0.f;
+  float zsum = p;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1)
+    zsum += __shfl_xor_sync(0xffffffffu, zsum, off);
+  if (lane < k) {
+    idx_out[t * k + lane] = my_e;
+    gate_out[t * k + lane] = p / zsum;
+  }
+  if (flags && lane == 0) {
+    const float margin = (k < E) ? kth_key - next_key : INFINITY;
+    flags[t] = (margin < 1e-4f) ? 1 : 0;
+  }
+}
+
+template <int PL>
+void launch_topk(const float* part, int nsplit, const float* bias,
+                 float* logits, int32_t* idx, float* gate, uint8_t* flags,
+                 int64_t T, int E, int k, cudaStream_t st) {
+  const int warps = 8;
+  const unsigned grid = (unsigned)((T + warps - 1) / warps);
+  topk_kernel<PL><<<grid, warps * 32, 0, st>>>(part, nsplit, bias, logits, idx,
+                                               gate, flags, T, E, k);
+}
+
+}  // namespace
+
+// Number of contraction splits so that the logits GEMM has >= ~2 CTAs per SM.
+int router_splits(const Shape& sh) {
+  const int64_t tiles = ((sh.E + RE - 1) / RE) * ((sh.T + RT - 1) / RT);
+  int64_t want = (296 + tiles - 1) / tiles;
+  const int64_t max_split = (sh.d + 255) / 256;  // >= 256 k per split
+  if (want > max_split) want = max_split;
+  if (want < 1) want = 1;
+  return (int)want;
+}
+
+cudaError_t launch_router(const Shape& sh, const void* x, const float* w_r,
+                          const float* bias, float* part, int32_t* idx,
+                          float* gate, uint8_t* flags, float* logits_out,
+                          cudaStream_t st) {
+  const int nsplit = router_splits(sh);
+  int64_t kps = (sh.d + nsplit - 1) / nsplit;
+  kps = (kps + RK - 1) / RK * RK;
+  dim3 grid((unsigned)((sh.E + RE - 1) / RE), (unsigned)((sh.T + RT - 1) / RT),
+            (unsigned)nsplit);
+  if (sh.bf16)
+    router_logits_kernel<__nv_bfloat16><<<grid, kRouterThreads, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(x), w_r, part, sh.T, sh.d, sh.E, kps);
+  else
+    router_logits_kernel<float><<<grid, kRouterThreads, 0, st>>>(
+        static_cast<const float*>(x), w_r, part, sh.T, sh.d, sh.E, kps);
+  const int pl = (int)((sh.E + 31) / 32);
+  const int E = (int)sh.E, k = (int)sh.k;
+  if (pl <= 1)
+    launch_topk<1>(part, nsplit, bias, logits_out, idx, gate, flags, sh.T, E, k, st);
+  else if (pl <= 2)
+    launch_topk<2>(part, nsplit, bias, logits_out, idx, gate, flags, sh.T, E, k, st);
+  else if (pl <= 4)
+    launch_topk<4>(part, nsplit, bias, logits_out, idx, gate, flags, sh.T, E, k, st);
+  else if (pl <= 8)
+    launch_topk<8>(part, nsplit, bias, logits_out, idx, gate, flags, sh.T, E, k, st);
+  else if (pl <= 16)
+    launch_topk<16>(part, nsplit, bias, logits_out, idx, gate, flags, sh.T, E, k, st);
+  else
+    launch_topk<32>(part, nsplit, bias, logits_out, idx, gate, flags, sh.T, E, k, st);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

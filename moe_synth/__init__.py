@@ -191,16 +191,32 @@ def make_expert(shape: MoEShape, seed: int, e: int):
     return wg, wu, wd
 
 
+_expert_cache: dict = {}
+
+
+def make_experts(shape: MoEShape, seed: int):
+    """All routed experts' weights. They depend only on (seed, N, F, d, dtype),
+    so layers that differ only in T or routing share them; the last set drawn
+    is kept (read-only use)."""
+    key = (seed, shape.n_routed, shape.ffn, shape.d, shape.act_dtype)
+    if key in _expert_cache:
+        return _expert_cache[key]
+    _expert_cache.clear()
+    dt = torch_dtype(shape.act_dtype)
+    N, F, d = shape.n_routed, shape.ffn, shape.d
+    wg = torch.empty(N, F, d, dtype=dt)
+    wu = torch.empty(N, F, d, dtype=dt)
+    wd = torch.empty(N, d, F, dtype=dt)
+    for e in range(N):
+        wg[e], wu[e], wd[e] = make_expert(shape, seed, e)
+    _expert_cache[key] = (wg, wu, wd)
+    return wg, wu, wd
+
+
 def make_inputs(shape: MoEShape, seed: int = 0, with_experts: bool = True,
                 beta: Optional[float] = None) -> Inputs:
     x, w_r, b = make_router_inputs(shape, seed, beta)
     wg = wu = wd = None
     if with_experts:
-        dt = torch_dtype(shape.act_dtype)
-        N, F, d = shape.n_routed, shape.ffn, shape.d
-        wg = torch.empty(N, F, d, dtype=dt)
-        wu = torch.empty(N, F, d, dtype=dt)
-        wd = torch.empty(N, d, F, dtype=dt)
-        for e in range(N):
-            wg[e], wu[e], wd[e] = make_expert(shape, seed, e)
+        wg, wu, wd = make_experts(shape, seed)
     return Inputs(shape, seed, x, w_r, b, wg, wu, wd)

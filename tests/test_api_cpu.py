@@ -1,0 +1,121 @@
+"""Host-side tests of the C ABI: the library builds for sm_100a, loads, exports
+every function the header declares, sizes its workspace, and rejects bad
+arguments on the host before anything would be launched (so these run without
+a GPU: no call here reaches a kernel launch)."""
+import ctypes
+
+import pytest
+
+import expert_routing_dispatch_router_b200 as moe
+from expert_routing_dispatch_router_b200 import build as moe_build
+
+P = ctypes.c_void_p
+
+
+@pytest.fixture(scope="module")
+def L():
+    moe_build.build()
+    return moe.lib()
+
+
+def cfg(T=64, d=256, N=8, Z=2, k=2, F=512, dt=moe.MOE_BF16, s=1.0):
+    return moe.MoEConfig(T, d, N, Z, k, F, dt, s)
+
+
+def test_every_declared_function_is_exported(L):
+    names = moe.declared_functions()
+    assert {"moe_route", "moe_dispatch", "moe_expert_ffn", "moe_combine",
+            "moe_layer_forward", "moe_workspace_size", "moe_status_string",
+            "moe_layer_forward_host", "moe_read_device_error",
+            "moe_layer_launch_count"} <= set(names)
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings(L):
+    for code in range(6):
+        assert L.moe_status_string(code)
+    assert L.moe_status_string(0) == b"ok"
+
+
+def test_workspace_size_valid_and_invalid(L):
+    c = cfg()
+    n = L.moe_workspace_size(ctypes.byref(c))
+    assert n > 0 and n % 1024 == 0
+    big = cfg(T=16384, d=4096, N=128, Z=32, k=8, F=1024)
+    nb = L.moe_workspace_size(ctypes.byref(big))
+    # holds at least x_perm, h and y_perm for T*k rows
+    assert nb >= 16384 * 8 * (4096 * 2 + 1024) * 2
+    for bad in (cfg(k=0), cfg(k=11), cfg(d=0), cfg(T=-1), cfg(N=0, Z=0),
+                cfg(dt=7), cfg(k=33, N=40), cfg(N=1020, Z=10), cfg(d=260),
+                cfg(F=100), cfg(s=float("inf"))):
+        assert L.moe_workspace_size(ctypes.byref(bad)) == 0
+    assert L.moe_workspace_size(None) == 0
+
+
+def test_launch_count(L):
+    assert L.moe_layer_launch_count(ctypes.byref(cfg())) == 2 + 4 + 3 + 1
+    assert L.moe_layer_launch_count(ctypes.byref(cfg(dt=moe.MOE_F32))) == 2 + 4 + 2 + 1
+    assert L.moe_layer_launch_count(ctypes.byref(cfg(T=0))) == 0
+
+
+def _fake(addr=0x10000):
+    return P(addr)
+
+
+def test_config_errors_before_launch(L):
+    st = P(0)
+    bad = [(cfg(k=11), 1), (cfg(k=33, N=40), 2), (cfg(N=1100, Z=0), 2),
+           (cfg(d=12), 2), (cfg(F=20), 2), (cfg(T=-5), 1), (cfg(dt=3), 1),
+           (cfg(N=0, Z=0), 1), (cfg(s=float("nan")), 1)]
+    for c, want in bad:
+        r = L.moe_route(ctypes.byref(c), _fake(), _fake(), _fake(), None, _fake(),
+                        _fake(), None, _fake(), 1 << 40, st)
+        assert r == want, (c.T, c.d, c.top_k, r)
+        r = L.moe_layer_forward(ctypes.byref(c), _fake(), _fake(), _fake(), _fake(),
+                                _fake(), _fake(), _fake(), None, _fake(), 1 << 40, st)
+        assert r == want
+    assert L.moe_route(None, _fake(), _fake(), _fake(), None, _fake(), _fake(), None,
+                       _fake(), 1 << 40, st) == 1
+
+
+def test_pointer_errors_before_launch(L):
+    c = cfg()
+    st = P(0)
+    ws_n = L.moe_workspace_size(ctypes.byref(c))
+    ok = [_fake(0x10000 + 0x100 * i) for i in range(12)]
+    # null required pointer
+    r = L.moe_layer_forward(ctypes.byref(c), None, *ok[1:7], None, ok[8], ws_n, st)
+    assert r == 1
+    # misaligned pointer
+    r = L.moe_layer_forward(ctypes.byref(c), _fake(0x10008), *ok[1:7], None, ok[8],
+                            ws_n, st)
+    assert r == 1
+    # misaligned optional pointer
+    r = L.moe_layer_forward(ctypes.byref(c), *ok[0:7], _fake(0x10004), ok[8], ws_n, st)
+    assert r == 1
+    # workspace missing / too small / misaligned base
+    r = L.moe_layer_forward(ctypes.byref(c), *ok[0:7], None, None, ws_n, st)
+    assert r == 3
+    r = L.moe_layer_forward(ctypes.byref(c), *ok[0:7], None, ok[8], ws_n - 1, st)
+    assert r == 3
+    r = L.moe_layer_forward(ctypes.byref(c), *ok[0:7], None, _fake(0x10010), ws_n, st)
+    assert r == 1
+    # staged calls
+    assert L.moe_dispatch(ctypes.byref(c), ok[0], None, *ok[2:7], ok[8], ws_n, st) == 1
+    assert L.moe_expert_ffn(ctypes.byref(c), ok[0], ok[1], None, ok[3], ok[4], ok[5],
+                            ok[8], ws_n, st) == 1
+    assert L.moe_combine(ctypes.byref(c), *ok[0:5], _fake(0x10001), ok[6], st) == 1
+    assert L.moe_expert_ffn(ctypes.byref(c), *ok[0:6], ok[8], 16, st) == 3
+    # host entry point: host pointers may be null-checked only
+    assert L.moe_layer_forward_host(ctypes.byref(c), None, *ok[1:6], ok[6], None,
+                                    ok[8], ws_n, st) == 1
+    assert L.moe_read_device_error(None, None, st) == 3
+
+
+def test_python_binding_marshalling_checks():
+    import torch
+    sh = moe.LayerShape(T=4, d=64, n_routed=2, n_zero=1, top_k=2, ffn=64)
+    x = torch.zeros(4, 64, dtype=torch.float32)
+    with pytest.raises(ValueError):
+        moe.route(sh, x, torch.zeros(3, 64), torch.zeros(3), ws=torch.zeros(1))

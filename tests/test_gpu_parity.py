@@ -1,0 +1,177 @@
+"""GPU parity: every stage of the CUDA library against the CPU oracle on the
+same seeded inputs, through the C ABI (Python binding = marshalling only).
+
+Staged calls are fed the ORACLE's outputs of the previous stage (never the
+GPU's), so each stage is compared on identical inputs. The fused layer is
+compared end to end. Small cases span several tiles and ragged tails; the
+named workloads run at full size, with the expert FFN checked on a seeded
+sample of tokens/rows that the oracle computes one by one.
+"""
+import numpy as np
+import pytest
+import torch
+
+import expert_routing_dispatch_router_b200 as moe
+import oracle
+from moe_synth import CONFIGS, MoEShape, get_config, make_inputs, torch_dtype
+from parity_helpers import (OUT_RTOL_RMS, alternative_selection, assert_logits_close,
+                            compare_selection, rel_rms_err)
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def layer_shape(sh: MoEShape, s=None) -> moe.LayerShape:
+    return moe.LayerShape(sh.T, sh.d, sh.n_routed, sh.n_zero, sh.top_k, sh.ffn,
+                          torch_dtype(sh.act_dtype),
+                          sh.routed_scale if s is None else s)
+
+
+SMALL = [
+    # several 128-row token tiles and ragged tails; F, d multiples of 128 -> tcgen05
+    MoEShape("small_bf16", T=300, d=256, n_routed=6, n_zero=2, top_k=3, ffn=384),
+    # skewed: one expert gets most tokens (multiple token tiles per expert)
+    MoEShape("skew_bf16", T=517, d=384, n_routed=5, n_zero=3, top_k=2, ffn=256,
+             routing="zipf"),
+    # d, F not multiples of 128 -> CUDA-core path in bf16
+    MoEShape("odd_bf16", T=77, d=200, n_routed=4, n_zero=1, top_k=2, ffn=136),
+    CONFIGS["tiny_fp32"],
+]
+
+
+def run_staged_and_fused(sh: MoEShape, seed: int, sample=None, s=None):
+    inp = make_inputs(sh, seed)
+    ls = layer_shape(sh, s)
+    scale = ls.routed_scale
+    d_inp = inp.to(DEV)
+    ws = moe.alloc_workspace(ls)
+    T, k, N, E = sh.T, sh.top_k, sh.n_routed, sh.E
+
+    # ---- router
+    ref_logits, ref_idx, ref_gate, ref_margin = oracle.route(inp.x, inp.w_router,
+                                                             inp.bias, k)
+    logits = torch.empty(T, E, dtype=torch.float32, device=DEV)
+    flags = torch.empty(T, dtype=torch.uint8, device=DEV)
+    g_idx, g_gate = moe.route(ls, d_inp.x, d_inp.w_router, d_inp.bias, ws,
+                              logits=logits, flags=flags)
+    torch.cuda.synchronize()
+    assert_logits_close(logits, ref_logits)
+    flagged = compare_selection(g_idx, g_gate, ref_idx, ref_gate, ref_margin,
+                                ref_logits, inp.bias, k)
+    fl = flags.cpu().numpy().astype(bool)
+    assert not np.any(fl & (ref_margin >= 2 * 1e-4)), "GPU flags a clear margin"
+    assert np.all(fl[ref_margin < 5e-5]), "GPU misses a near tie"
+
+    # ---- dispatch, fed the oracle's selection
+    r_counts, r_offsets, r_row_token, r_slot_row = oracle.dispatch(ref_idx, N, E)
+    R = int(r_offsets[N])
+    counts, offsets, row_token, slot_row, x_perm = moe.dispatch(
+        ls, d_inp.x, torch.from_numpy(ref_idx).to(DEV), ws)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(counts.cpu().numpy(), r_counts)
+    np.testing.assert_array_equal(offsets.cpu().numpy(), r_offsets)
+    np.testing.assert_array_equal(row_token.cpu().numpy(), r_row_token)
+    np.testing.assert_array_equal(slot_row.cpu().numpy(), r_slot_row)
+    assert torch.equal(x_perm[:R].cpu(), inp.x[torch.from_numpy(r_row_token[:R]).long()])
+
+    # ---- expert FFN, fed the oracle's dispatch
+    x_perm_ref = torch.zeros(T * k, sh.d, dtype=inp.x.dtype)
+    x_perm_ref[:R] = inp.x[torch.from_numpy(r_row_token[:R]).long()]
+    y_perm = moe.expert_ffn(ls, x_perm_ref.to(DEV), torch.from_numpy(r_offsets).to(DEV),
+                            d_inp.w_gate, d_inp.w_up, d_inp.w_down, ws)
+    torch.cuda.synchronize()
+    row_expert = np.repeat(np.arange(N), r_counts[:N]).astype(np.int32)
+    rows = np.arange(R) if sample is None else np.unique(
+        np.random.default_rng(seed).choice(R, size=min(sample, R), replace=False))
+    if R > 0:
+        y_ref = oracle.expert_rows(inp.w_gate, inp.w_up, inp.w_down, row_expert[rows],
+                                   x_perm_ref[torch.from_numpy(rows).long()])
+        got = y_perm[torch.from_numpy(rows).long().to(DEV)].double().cpu().numpy()
+        err = rel_rms_err(got, y_ref)
+        assert err <= OUT_RTOL_RMS, f"expert rows: max err {err:.3e} x rms"
+
+    # ---- combine, fed the oracle's gates and expert outputs (rounded to act dtype)
+    tok = np.arange(T) if sample is None else np.unique(
+        np.random.default_rng(seed + 7).choice(T, size=min(sample, T), replace=False))
+    if sample is None and R > 0:
+        y_all = oracle.expert_rows(inp.w_gate, inp.w_up, inp.w_down, row_expert,
+                                   x_perm_ref[:R])
+        y_in = torch.zeros(T * k, sh.d, dtype=inp.x.dtype)
+        y_in[:R] = torch.from_numpy(y_all).to(inp.x.dtype)
+        gate32 = torch.from_numpy(ref_gate).float()
+        out_c = moe.combine(ls, d_inp.x, y_in.to(DEV), torch.from_numpy(ref_idx).to(DEV),
+                            gate32.to(DEV), torch.from_numpy(r_slot_row).to(DEV))
+        torch.cuda.synchronize()
+        ref_c = oracle.combine(inp.x, y_in, ref_idx, gate32, r_slot_row, N, scale)
+        err = rel_rms_err(out_c.double().cpu().numpy(), ref_c)
+        assert err <= 1e-2, f"combine: max err {err:.3e} x rms"
+
+    # ---- fused layer
+    out = torch.empty(T, sh.d, dtype=inp.x.dtype, device=DEV)
+    g_counts = torch.empty(E, dtype=torch.int32, device=DEV)
+    moe.layer_forward(ls, d_inp.x, d_inp.w_router, d_inp.bias, d_inp.w_gate,
+                      d_inp.w_up, d_inp.w_down, ws, out=out, counts=g_counts)
+    torch.cuda.synchronize()
+    assert moe.read_device_error(ws) == 0
+    gc = g_counts.cpu().numpy()
+    assert gc.sum() == T * k
+    if not flagged.any():
+        np.testing.assert_array_equal(gc, r_counts)
+    else:
+        assert np.abs(gc - r_counts).sum() <= 2 * int(flagged.sum())
+    out_ref, _, _ = oracle.layer(inp.x, inp.w_router, inp.bias, inp.w_gate, inp.w_up,
+                                 inp.w_down, N, k, scale, tokens=tok.astype(np.int32))
+    got = out[torch.from_numpy(tok).long().to(DEV)].double().cpu().numpy()
+    keep = ~flagged[tok]
+    err = rel_rms_err(got[keep], out_ref[keep])
+    assert err <= OUT_RTOL_RMS, f"layer: max err {err:.3e} x rms"
+    # near-tied tokens must match one of the valid answers
+    for n in np.nonzero(~keep)[0]:
+        t = int(tok[n])
+        alt = ref_idx.copy()
+        alt[t] = alternative_selection(ref_logits[t], inp.bias, k)
+        alt_out, _, _ = oracle.layer(inp.x, inp.w_router, inp.bias, inp.w_gate,
+                                     inp.w_up, inp.w_down, N, k, scale,
+                                     tokens=np.array([t], np.int32), force_idx=alt)
+        e1 = rel_rms_err(got[n:n + 1], out_ref[n:n + 1])
+        e2 = rel_rms_err(got[n:n + 1], alt_out)
+        assert min(e1, e2) <= OUT_RTOL_RMS
+    # deterministic: a second run is bit-identical
+    out2 = torch.empty_like(out)
+    moe.layer_forward(ls, d_inp.x, d_inp.w_router, d_inp.bias, d_inp.w_gate,
+                      d_inp.w_up, d_inp.w_down, ws, out=out2)
+    torch.cuda.synchronize()
+    assert torch.equal(out, out2)
+    return {"flagged": int(flagged.sum()), "R": R}
+
+
+@pytest.mark.parametrize("sh", SMALL, ids=lambda s: s.name)
+@pytest.mark.parametrize("seed", [0, 1])
+def test_small_configs(sh, seed):
+    run_staged_and_fused(sh, seed)
+
+
+def test_routed_scale_nine():
+    run_staged_and_fused(SMALL[0], 2, s=9.0)
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_decode_full(seed):
+    run_staged_and_fused(CONFIGS["decode"], seed)
+
+
+def test_prefill_full_sampled():
+    run_staged_and_fused(CONFIGS["prefill"], 0, sample=48)
+
+
+def test_large_e_full_sampled():
+    info = run_staged_and_fused(CONFIGS["large_e"], 0, sample=24)
+    sh = CONFIGS["large_e"]
+    zero_share = 1.0 - info["R"] / (sh.T * sh.top_k)
+    assert 0.29 <= zero_share <= 0.31
+
+
+@pytest.mark.parametrize("T", [1, 8, 64])
+def test_sweep_small_T(T):
+    run_staged_and_fused(get_config(f"sweep_uniform_T{T}"), 0)
