@@ -10,9 +10,9 @@
 //   out[t] = s * sum_{j: idx<N} gate[t,j] * y_perm[slot_row[t,j]]
 //              + sum_{j: idx>=N} gate[t,j] * x[t]
 //
-// Both sums run in fp32 in slot order j = 0..k-1 and the result is rounded
-// once, so the output does not depend on thread timing. Grid: one block row
-// per token, 16-byte vectors along d.
+// y_perm is fp32. Both sums run in fp32 in slot order j = 0..k-1 and the
+// result is rounded once, so the output does not depend on thread timing.
+// Grid: one block row per token, 16-byte vectors along d.
 #include "moe_internal.cuh"
 
 namespace moe {
@@ -59,7 +59,7 @@ struct Vec<float> {
 
 template <typename AT>
 __global__ void __launch_bounds__(128)
-    combine_kernel(const AT* __restrict__ x, const AT* __restrict__ y,
+    combine_kernel(const AT* __restrict__ x, const float* __restrict__ y,
                    const int32_t* __restrict__ idx,
                    const float* __restrict__ gate,
                    const int32_t* __restrict__ slot_row, AT* __restrict__ out,
@@ -68,6 +68,8 @@ __global__ void __launch_bounds__(128)
   __shared__ int32_t s_row[kMaxTopK];
   __shared__ float s_gate[kMaxTopK];
   __shared__ int32_t s_zero[kMaxTopK];
+  griddep_wait();
+  griddep_launch_dependents();
   const int64_t t = blockIdx.x;
   if (threadIdx.x < k) {
     const int e = idx[t * k + threadIdx.x];
@@ -95,7 +97,8 @@ __global__ void __launch_bounds__(128)
     } else {
       const int64_t r = s_row[j];
       if (r < 0) continue;
-      Vec<AT>::load(y + r * d + col, v);
+#pragma unroll
+      for (int i = 0; i < V; i += 4) Vec<float>::load(y + r * d + col + i, v + i);
 #pragma unroll
       for (int i = 0; i < V; ++i) racc[i] = fmaf(g, v[i], racc[i]);
     }
@@ -115,15 +118,15 @@ cudaError_t launch_combine(const Shape& sh, const void* x, const void* y_perm,
   const int threads = 128;
   dim3 grid((unsigned)sh.T, (unsigned)((vecs + threads - 1) / threads));
   if (sh.bf16)
-    combine_kernel<__nv_bfloat16><<<grid, threads, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(x),
-        static_cast<const __nv_bfloat16*>(y_perm), idx, gate, slot_row,
-        static_cast<__nv_bfloat16*>(out), sh.d, (int)sh.N, (int)sh.k, sh.s);
+    launch_pdl(combine_kernel<__nv_bfloat16>, grid, dim3(threads), 0, st,
+               static_cast<const __nv_bfloat16*>(x), static_cast<const float*>(y_perm),
+               idx, gate, slot_row, static_cast<__nv_bfloat16*>(out), sh.d, (int)sh.N,
+               (int)sh.k, sh.s);
   else
-    combine_kernel<float><<<grid, threads, 0, st>>>(
-        static_cast<const float*>(x), static_cast<const float*>(y_perm), idx,
-        gate, slot_row, static_cast<float*>(out), sh.d, (int)sh.N, (int)sh.k,
-        sh.s);
+    launch_pdl(combine_kernel<float>, grid, dim3(threads), 0, st,
+               static_cast<const float*>(x), static_cast<const float*>(y_perm), idx,
+               gate, slot_row, static_cast<float*>(out), sh.d, (int)sh.N, (int)sh.k,
+               sh.s);
   return cudaGetLastError();
 }
 

@@ -8,7 +8,9 @@
 // the same on every run (the deterministic operators of "LongCat-2.0 Derruba
 // Dois Tetos", section "A Primeira Parede").
 //
-// Three small kernels plus a gather, no atomics whose order matters:
+// For small batches (the masks of all T tokens fit in shared memory) one block
+// does steps 1-3 in a single launch (dispatch_small_kernel). Otherwise three
+// small kernels plus the gather, no atomics whose order matters:
 //  1. dispatch_count_kernel: each block takes 256 tokens and builds, in shared
 //     memory, one 256-bit mask per expert (which of its tokens chose it), then
 //     writes popcount(mask) = the block's count per expert.
@@ -61,6 +63,8 @@ __global__ void __launch_bounds__(kChunkTokens)
                           int E, int32_t* __restrict__ chunk_base,
                           int32_t* err) {
   extern __shared__ uint32_t mask[];
+  griddep_wait();
+  griddep_launch_dependents();
   build_masks(mask, idx, T, k, E, err);
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     int c = 0;
@@ -77,6 +81,8 @@ __global__ void __launch_bounds__(1024)
                          int32_t* __restrict__ row_token, int64_t rows_cap) {
   __shared__ int32_t warp_sums[32];
   __shared__ int32_t total_s;
+  griddep_wait();
+  griddep_launch_dependents();
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     int32_t run = 0;
     for (int64_t c = 0; c < nchunks; ++c) {
@@ -124,6 +130,8 @@ __global__ void __launch_bounds__(kChunkTokens)
                             int32_t* __restrict__ row_token,
                             int32_t* __restrict__ slot_row) {
   extern __shared__ uint32_t mask[];
+  griddep_wait();
+  griddep_launch_dependents();
   build_masks(mask, idx, T, k, E, nullptr);
   const int64_t t = (int64_t)blockIdx.x * kChunkTokens + threadIdx.x;
   if (t >= T) return;
@@ -142,6 +150,100 @@ __global__ void __launch_bounds__(kChunkTokens)
   }
 }
 
+// Block-wide exclusive scan of v over threads (blockDim.x == 1024). Returns
+// the sum of the values before this thread; *total gets the sum of all.
+__device__ __forceinline__ int32_t block_exclusive_scan(int32_t v, int32_t* warp_sums,
+                                                        int32_t* total) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  int32_t incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int32_t o = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += o;
+  }
+  if (lane == 31) warp_sums[wid] = incl;
+  __syncthreads();
+  if (wid == 0) {
+    int32_t s = warp_sums[lane];
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int32_t o = __shfl_up_sync(0xffffffffu, s, off);
+      if (lane >= off) s += o;
+    }
+    warp_sums[lane] = s;
+  }
+  __syncthreads();
+  *total = warp_sums[31];
+  return (wid > 0 ? warp_sums[wid - 1] : 0) + incl - v;
+}
+
+// Steps 1-3 in one block for a batch whose masks fit in shared memory:
+// mask[e*W + w] bit b = token 32w + b chose e; pre[e*W + w] = set bits of
+// expert e in words before w. rank of token t in expert e = pre + bits below t.
+__global__ void __launch_bounds__(1024)
+    dispatch_small_kernel(const int32_t* __restrict__ idx, int T, int k, int E, int N,
+                          int W, int32_t* __restrict__ counts,
+                          int32_t* __restrict__ offsets, int32_t* __restrict__ row_token,
+                          int32_t* __restrict__ slot_row, int64_t rows_cap,
+                          int32_t* err) {
+  extern __shared__ uint32_t sm[];
+  uint32_t* mask = sm;
+  int32_t* pre = reinterpret_cast<int32_t*>(sm + (size_t)E * W);
+  int32_t* s_off = pre + (size_t)E * W;
+  __shared__ int32_t warp_sums[32];
+  griddep_wait();
+  griddep_launch_dependents();
+  for (int i = threadIdx.x; i < E * W; i += blockDim.x) mask[i] = 0u;
+  __syncthreads();
+  for (int t = threadIdx.x; t < T; t += blockDim.x) {
+    const uint32_t bit = 1u << (t & 31);
+    for (int j = 0; j < k; ++j) {
+      const int e = idx[(int64_t)t * k + j];
+      if (e < 0 || e >= E) {
+        record_error(err, kErrBadExpertId);
+        continue;
+      }
+      const uint32_t old = atomicOr(&mask[e * W + (t >> 5)], bit);
+      if (old & bit) record_error(err, kErrBadExpertId);
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int32_t run = 0;
+    for (int w = 0; w < W; ++w) {
+      pre[e * W + w] = run;
+      run += __popc(mask[e * W + w]);
+    }
+    counts[e] = run;
+    if (e < N) s_off[e] = run;
+  }
+  __syncthreads();
+  int32_t R = 0;
+  const int32_t v = ((int)threadIdx.x < N) ? s_off[threadIdx.x] : 0;
+  const int32_t before = block_exclusive_scan(v, warp_sums, &R);
+  __syncthreads();
+  if ((int)threadIdx.x < N) {
+    s_off[threadIdx.x] = before;
+    offsets[threadIdx.x] = before;
+  }
+  if (threadIdx.x == 0) offsets[N] = R;
+  __syncthreads();
+  for (int t = threadIdx.x; t < T; t += blockDim.x) {
+    const int w = t >> 5;
+    const uint32_t below = (1u << (t & 31)) - 1u;
+    for (int j = 0; j < k; ++j) {
+      const int e = idx[(int64_t)t * k + j];
+      int32_t r = -1;
+      if (e >= 0 && e < N) {
+        r = s_off[e] + pre[e * W + w] + __popc(mask[e * W + w] & below);
+        row_token[r] = t;
+      }
+      slot_row[(int64_t)t * k + j] = r;
+    }
+  }
+  for (int64_t r = R + threadIdx.x; r < rows_cap; r += blockDim.x) row_token[r] = -1;
+}
+
 // x_perm[r, :] = x[row_token[r], :] for r < R; one warp per row, 16-byte vectors.
 __global__ void __launch_bounds__(256)
     gather_rows_kernel(const uint4* __restrict__ x,
@@ -149,6 +251,8 @@ __global__ void __launch_bounds__(256)
                        const int32_t* __restrict__ offsets, int N,
                        int64_t vec_per_row, int64_t rows_cap,
                        uint4* __restrict__ x_perm) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int64_t R = offsets[N];
   const int lane = threadIdx.x & 31;
   const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
@@ -162,6 +266,21 @@ __global__ void __launch_bounds__(256)
 }
 
 }  // namespace
+
+constexpr size_t kSmallDispatchSmem = 96 * 1024;
+
+size_t dispatch_small_smem(const Shape& sh) {
+  const size_t W = (size_t)((sh.T + 31) / 32);
+  return (2 * (size_t)sh.E * W + (size_t)sh.N) * sizeof(uint32_t);
+}
+
+bool dispatch_small_fits(const Shape& sh) {
+  return sh.T <= 4096 && dispatch_small_smem(sh) <= kSmallDispatchSmem;
+}
+
+int dispatch_launch_count(const Shape& sh) {
+  return (dispatch_small_fits(sh) ? 1 : 3) + (sh.N > 0 ? 1 : 0);
+}
 
 int num_sms() {
   static int n = 0;
@@ -180,14 +299,34 @@ cudaError_t launch_dispatch(const Shape& sh, const void* x, const int32_t* idx,
                             int32_t* slot_row, void* x_perm, int32_t* err,
                             cudaStream_t st) {
   const int E = (int)sh.E, N = (int)sh.N, k = (int)sh.k;
-  const size_t smem = (size_t)E * kWords * sizeof(uint32_t);
-  const unsigned nch = (unsigned)sh.nchunks;
-  dispatch_count_kernel<<<nch, kChunkTokens, smem, st>>>(idx, sh.T, k, E,
-                                                         chunk_base, err);
-  dispatch_scan_kernel<<<1, 1024, 0, st>>>(chunk_base, sh.nchunks, E, N, counts,
-                                           offsets, row_token, sh.T * sh.k);
-  dispatch_scatter_kernel<<<nch, kChunkTokens, smem, st>>>(
-      idx, sh.T, k, E, N, chunk_base, offsets, row_token, slot_row);
+  cudaError_t e = cudaSuccess;
+  if (dispatch_small_fits(sh)) {
+    const int W = (int)((sh.T + 31) / 32);
+    const size_t smem = dispatch_small_smem(sh);
+    static bool attr_set = false;
+    if (!attr_set) {
+      e = cudaFuncSetAttribute(dispatch_small_kernel,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)kSmallDispatchSmem);
+      if (e != cudaSuccess) return e;
+      attr_set = true;
+    }
+    e = launch_pdl(dispatch_small_kernel, dim3(1), dim3(1024), smem, st, idx, (int)sh.T,
+                   k, E, N, W, counts, offsets, row_token, slot_row, sh.T * sh.k, err);
+    if (e != cudaSuccess) return e;
+  } else {
+    const size_t smem = (size_t)E * kWords * sizeof(uint32_t);
+    const unsigned nch = (unsigned)sh.nchunks;
+    e = launch_pdl(dispatch_count_kernel, dim3(nch), dim3(kChunkTokens), smem, st, idx,
+                   sh.T, k, E, chunk_base, err);
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(dispatch_scan_kernel, dim3(1), dim3(1024), 0, st, chunk_base,
+                   sh.nchunks, E, N, counts, offsets, row_token, sh.T * sh.k);
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(dispatch_scatter_kernel, dim3(nch), dim3(kChunkTokens), smem, st, idx,
+                   sh.T, k, E, N, chunk_base, offsets, row_token, slot_row);
+    if (e != cudaSuccess) return e;
+  }
   if (N > 0) {
     const int64_t vpr = sh.d * sh.es / 16;
     int64_t rows = sh.T * sh.k;
@@ -195,9 +334,10 @@ cudaError_t launch_dispatch(const Shape& sh, const void* x, const int32_t* idx,
     const int64_t cap = (int64_t)num_sms() * 8;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
-    gather_rows_kernel<<<(unsigned)blocks, 256, 0, st>>>(
-        static_cast<const uint4*>(x), row_token, offsets, N, vpr, rows,
-        static_cast<uint4*>(x_perm));
+    e = launch_pdl(gather_rows_kernel, dim3((unsigned)blocks), dim3(256), 0, st,
+                   static_cast<const uint4*>(x), row_token, offsets, N, vpr, rows,
+                   static_cast<uint4*>(x_perm));
+    if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
 }

@@ -28,9 +28,11 @@
 // error code in the workspace, the other roles stop, outstanding TMA loads and
 // MMAs are waited for (again bounded), TMEM is freed and the kernel returns.
 //
+// Rounding points: h is stored in the activation type (bf16 feeds the tensor
+// cores); y is written in fp32 so that the combine rounds the output only once.
+//
 // CUDA-core path (f32, or shapes the tensor-core path does not take): one warp
-// per output element, fp32 accumulation, same rounding points (h is stored in
-// the activation type).
+// per output element, fp32 accumulation, same rounding points.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -47,6 +49,8 @@ __global__ void __launch_bounds__(1024)
     gemm_plan_kernel(const int32_t* __restrict__ offsets, int N,
                      int32_t* __restrict__ tile_start) {
   __shared__ int32_t warp_sums[32];
+  griddep_wait();
+  griddep_launch_dependents();
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   int32_t v = 0;
   if ((int)threadIdx.x < N) {
@@ -100,7 +104,7 @@ struct Cfg {
 struct GemmArgs {
   const int32_t* offsets;     // [N+1] row offsets per expert
   const int32_t* tile_start;  // [N+1] token-tile prefix per expert
-  __nv_bfloat16* out;         // [rows_cap, out_cols]
+  void* out;                  // [rows_cap, out_cols]: bf16 h or fp32 y
   int32_t* err;               // workspace error word
   int N;
   int num_kb;    // contraction length / BK
@@ -191,10 +195,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int N = args.N;
-  for (int i = threadIdx.x; i <= N; i += blockDim.x) {
-    s_tiles[i] = args.tile_start[i];
-    s_offs[i] = args.offsets[i];
-  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       ptx::mbar_init(full_bar(s), 1);
@@ -217,6 +217,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     ptx::tmem_alloc(ptx::smem_addr(tmem_slot), kTmemCols);
     ptx::tmem_relinquish();
+  }
+  // everything above overlaps the previous kernel's tail; the plan and the
+  // operands are read only after it has completed
+  griddep_wait();
+  griddep_launch_dependents();
+  for (int i = threadIdx.x; i <= N; i += blockDim.x) {
+    s_tiles[i] = args.tile_start[i];
+    s_offs[i] = args.offsets[i];
   }
   ptx::tc_fence_before();
   __syncthreads();
@@ -330,19 +338,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(ew * 32) << 16) +
                           (uint32_t)acc * kAccStride;
       const int64_t col = (int64_t)un.m * BM + lrow;
-      __nv_bfloat16* outp = args.out + (int64_t)un.row0 * args.out_cols + col;
+      const int64_t obase = (int64_t)un.row0 * args.out_cols + col;
       for (int c0 = 0; c0 < un.n_mma; c0 += 16) {
         float g[16], v[16];
-        if (GATEUP)
+        if (GATEUP) {
           ptx::tmem_ld16x2(tb + c0, tb + 128 + c0, g, v);
-        else
-          ptx::tmem_ld16(tb + c0, g);
+          __nv_bfloat16* outp = static_cast<__nv_bfloat16*>(args.out) + obase;
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          if (c0 + c < un.n_valid) {
-            const float r = GATEUP ? silu_f(g[c]) * v[c] : g[c];
-            outp[(int64_t)(c0 + c) * args.out_cols] = __float2bfloat16_rn(r);
-          }
+          for (int c = 0; c < 16; ++c)
+            if (c0 + c < un.n_valid)
+              outp[(int64_t)(c0 + c) * args.out_cols] =
+                  __float2bfloat16_rn(silu_f(g[c]) * v[c]);
+        } else {
+          ptx::tmem_ld16(tb + c0, g);
+          float* outp = static_cast<float*>(args.out) + obase;
+#pragma unroll
+          for (int c = 0; c < 16; ++c)
+            if (c0 + c < un.n_valid) outp[(int64_t)(c0 + c) * args.out_cols] = g[c];
         }
       }
       ptx::tc_fence_before();
@@ -403,9 +415,8 @@ cudaError_t launch_tc(const CUtensorMap& a0, const CUtensorMap& a1,
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  grouped_gemm_tc_kernel<GATEUP><<<num_sms(), kThreads, C::kSmemBytes, st>>>(
-      a0, a1, b16, b128, args);
-  return cudaGetLastError();
+  return launch_pdl(grouped_gemm_tc_kernel<GATEUP>, dim3(num_sms()), dim3(kThreads),
+                    C::kSmemBytes, st, a0, a1, b16, b128, args);
 }
 
 // --------------------------------------------------------- CUDA-core path --
@@ -434,6 +445,8 @@ __global__ void __launch_bounds__(256)
     ffn_gateup_simt_kernel(const AT* __restrict__ x, const int32_t* __restrict__ offsets,
                            int N, const AT* __restrict__ wg, const AT* __restrict__ wu,
                            AT* __restrict__ h, int64_t d, int64_t F) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int64_t R = offsets[N];
   const int lane = threadIdx.x & 31;
   const int64_t nw = (int64_t)gridDim.x * (blockDim.x >> 5);
@@ -456,12 +469,14 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// y[r, n] = h[r] . w_down[e, n]
+// y[r, n] = h[r] . w_down[e, n]   (y kept in fp32)
 template <typename AT>
 __global__ void __launch_bounds__(256)
     ffn_down_simt_kernel(const AT* __restrict__ h, const int32_t* __restrict__ offsets,
-                         int N, const AT* __restrict__ wd, AT* __restrict__ y,
+                         int N, const AT* __restrict__ wd, float* __restrict__ y,
                          int64_t d, int64_t F) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int64_t R = offsets[N];
   const int lane = threadIdx.x & 31;
   const int64_t nw = (int64_t)gridDim.x * (blockDim.x >> 5);
@@ -474,7 +489,7 @@ __global__ void __launch_bounds__(256)
     float acc = 0.f;
     for (int64_t f = lane; f < F; f += 32) acc = fmaf(to_f32(dr[f]), to_f32(hr[f]), acc);
     acc = warp_sum<AT>(acc);
-    if (lane == 0) y[r * d + n] = from_f32<AT>(acc);
+    if (lane == 0) y[r * d + n] = acc;
   }
 }
 
@@ -483,13 +498,14 @@ cudaError_t launch_simt(const Shape& sh, const void* x_perm, const int32_t* offs
                         const void* wg, const void* wu, const void* wd, void* h,
                         void* y, cudaStream_t st) {
   const unsigned blocks = (unsigned)num_sms() * 16;
-  ffn_gateup_simt_kernel<AT><<<blocks, 256, 0, st>>>(
-      static_cast<const AT*>(x_perm), offsets, (int)sh.N, static_cast<const AT*>(wg),
-      static_cast<const AT*>(wu), static_cast<AT*>(h), sh.d, sh.F);
-  ffn_down_simt_kernel<AT><<<blocks, 256, 0, st>>>(
-      static_cast<const AT*>(h), offsets, (int)sh.N, static_cast<const AT*>(wd),
-      static_cast<AT*>(y), sh.d, sh.F);
-  return cudaGetLastError();
+  cudaError_t e = launch_pdl(ffn_gateup_simt_kernel<AT>, dim3(blocks), dim3(256), 0, st,
+                             static_cast<const AT*>(x_perm), offsets, (int)sh.N,
+                             static_cast<const AT*>(wg), static_cast<const AT*>(wu),
+                             static_cast<AT*>(h), sh.d, sh.F);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(ffn_down_simt_kernel<AT>, dim3(blocks), dim3(256), 0, st,
+                    static_cast<const AT*>(h), offsets, (int)sh.N,
+                    static_cast<const AT*>(wd), static_cast<float*>(y), sh.d, sh.F);
 }
 
 }  // namespace
@@ -527,14 +543,14 @@ cudaError_t launch_expert_ffn(const Shape& sh, const void* x_perm,
       make_map(&h128, h, rows_cap, (uint64_t)sh.F, BN);
   if (!ok) return cudaErrorInvalidValue;
 
-  gemm_plan_kernel<<<1, 1024, 0, st>>>(offsets, (int)sh.N, tile_start);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(gemm_plan_kernel, dim3(1), dim3(1024), 0, st, offsets,
+                             (int)sh.N, tile_start);
   if (e != cudaSuccess) return e;
 
   GemmArgs gu;
   gu.offsets = offsets;
   gu.tile_start = tile_start;
-  gu.out = static_cast<__nv_bfloat16*>(h);
+  gu.out = h;
   gu.err = err;
   gu.N = (int)sh.N;
   gu.num_kb = (int)(sh.d / BK);
@@ -544,7 +560,7 @@ cudaError_t launch_expert_ffn(const Shape& sh, const void* x_perm,
   if (e != cudaSuccess) return e;
 
   GemmArgs dn = gu;
-  dn.out = static_cast<__nv_bfloat16*>(y_perm);
+  dn.out = y_perm;
   dn.num_kb = (int)(sh.F / BK);
   dn.out_cols = (int)sh.d;
   dn.m_tiles = (int)(sh.d / BM);

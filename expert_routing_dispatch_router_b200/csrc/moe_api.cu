@@ -34,7 +34,7 @@ WsLayout ws_layout(const Shape& sh) {
   L.tile_start = take((size_t)(sh.N + 1) * sizeof(int32_t));
   L.x_perm = take(Tk * sh.d * sh.es);
   L.h = take(Tk * sh.F * sh.es);
-  L.y_perm = take(Tk * sh.d * sh.es);
+  L.y_perm = take(Tk * sh.d * sizeof(float));
   L.x_stage = take((size_t)sh.T * sh.d * sh.es);
   L.out_stage = take((size_t)sh.T * sh.d * sh.es);
   L.total = off;
@@ -275,7 +275,7 @@ int32_t moe_layer_launch_count(const moe_config_t* cfg) {
   Shape sh;
   if (make_shape(cfg, &sh) != MOE_OK || sh.T == 0) return 0;
   int32_t n = 2;                  // router logits + top-k
-  n += 3 + (sh.N > 0 ? 1 : 0);    // count, scan, scatter (+ gather)
+  n += dispatch_launch_count(sh);  // (count, scan, scatter | small) + gather
   n += expert_ffn_launch_count(sh);
   n += 1;                         // combine
   return n;

@@ -6,6 +6,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/moe_api.h"
 
 namespace moe {
@@ -35,7 +37,7 @@ struct WsLayout {
   size_t tile_start;   // int32 [N + 1] (expert GEMM plan)
   size_t x_perm;       // act   [T*k, d]
   size_t h;            // act   [T*k, F]
-  size_t y_perm;       // act   [T*k, d]
+  size_t y_perm;       // float [T*k, d]
   size_t x_stage;      // act   [T, d]   (host-buffer entry point)
   size_t out_stage;    // act   [T, d]
   size_t total;
@@ -71,10 +73,40 @@ cudaError_t launch_combine(const Shape& sh, const void* x, const void* y_perm,
                            const int32_t* idx, const float* gate,
                            const int32_t* slot_row, void* out, cudaStream_t st);
 int expert_ffn_launch_count(const Shape& sh);
+int dispatch_launch_count(const Shape& sh);
 bool expert_ffn_uses_tensor_cores(const Shape& sh);
 int num_sms();
 
+// Launch with programmatic dependent launch allowed: the kernel may start
+// while its predecessor on the stream drains, and must call griddep_wait()
+// before it reads or writes anything the predecessor touches.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // ---- device helpers ----
+// Wait until the previous kernel on the stream has completed and its memory
+// is visible (no-op when launched without programmatic dependencies).
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+// Allow the next kernel on the stream to be scheduled.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ float bf16_to_f32(uint16_t b) {
   return __uint_as_float(static_cast<uint32_t>(b) << 16);
 }

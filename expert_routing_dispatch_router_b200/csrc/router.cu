@@ -31,56 +31,81 @@ constexpr int RE = 32;   // experts per CTA
 constexpr int RK = 32;   // contraction chunk
 constexpr int kRouterThreads = 256;
 
+// Register staging of one 64-token x 32-k chunk of x (converted to fp32 when
+// stored to shared memory) and one 32-expert x 32-k chunk of w_r.
 template <typename XT>
-__device__ __forceinline__ void load_x_chunk(const XT* x, int64_t T, int64_t d,
-                                             int64_t t0, int64_t k0,
-                                             int64_t kend,
-                                             float (*xs)[RT + 4]);
+struct XChunk;
 
 // bf16 x: 64 tokens x 32 k = 256 vectors of 8 elements, one per thread.
 template <>
-__device__ __forceinline__ void load_x_chunk<__nv_bfloat16>(
-    const __nv_bfloat16* x, int64_t T, int64_t d, int64_t t0, int64_t k0,
-    int64_t kend, float (*xs)[RT + 4]) {
-  const int tid = threadIdx.x;
-  const int tt = tid >> 2;
-  const int kk = (tid & 3) * 8;
-  const int64_t t = t0 + tt;
-  const int64_t k = k0 + kk;
-  uint4 v = make_uint4(0, 0, 0, 0);
-  if (t < T && k < kend)
-    v = *reinterpret_cast<const uint4*>(x + t * d + k);
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    xs[kk + 2 * i][tt] = __uint_as_float(w[i] << 16);
-    xs[kk + 2 * i + 1][tt] = __uint_as_float(w[i] & 0xffff0000u);
+struct XChunk<__nv_bfloat16> {
+  uint4 v;
+  __device__ __forceinline__ void load(const __nv_bfloat16* x, int64_t T, int64_t d,
+                                       int64_t t0, int64_t k0, int64_t kend) {
+    const int tt = threadIdx.x >> 2;
+    const int kk = (threadIdx.x & 3) * 8;
+    const int64_t t = t0 + tt, k = k0 + kk;
+    v = make_uint4(0, 0, 0, 0);
+    if (t < T && k < kend) v = *reinterpret_cast<const uint4*>(x + t * d + k);
   }
-}
+  __device__ __forceinline__ void store(float (*xs)[RT + 4]) const {
+    const int tt = threadIdx.x >> 2;
+    const int kk = (threadIdx.x & 3) * 8;
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      xs[kk + 2 * i][tt] = __uint_as_float(w[i] << 16);
+      xs[kk + 2 * i + 1][tt] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+  }
+};
 
 // f32 x: 64 tokens x 32 k = 512 vectors of 4 elements, two per thread.
 template <>
-__device__ __forceinline__ void load_x_chunk<float>(const float* x, int64_t T,
-                                                    int64_t d, int64_t t0,
-                                                    int64_t k0, int64_t kend,
-                                                    float (*xs)[RT + 4]) {
+struct XChunk<float> {
+  float4 v[2];
+  __device__ __forceinline__ void load(const float* x, int64_t T, int64_t d, int64_t t0,
+                                       int64_t k0, int64_t kend) {
 #pragma unroll
-  for (int rep = 0; rep < 2; ++rep) {
-    const int v_id = threadIdx.x + rep * kRouterThreads;
-    const int tt = v_id >> 3;
-    const int kk = (v_id & 7) * 4;
-    const int64_t t = t0 + tt;
-    const int64_t k = k0 + kk;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (t < T && k < kend) v = *reinterpret_cast<const float4*>(x + t * d + k);
-    xs[kk + 0][tt] = v.x;
-    xs[kk + 1][tt] = v.y;
-    xs[kk + 2][tt] = v.z;
-    xs[kk + 3][tt] = v.w;
+    for (int rep = 0; rep < 2; ++rep) {
+      const int v_id = threadIdx.x + rep * kRouterThreads;
+      const int64_t t = t0 + (v_id >> 3), k = k0 + (v_id & 7) * 4;
+      v[rep] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (t < T && k < kend) v[rep] = *reinterpret_cast<const float4*>(x + t * d + k);
+    }
   }
-}
+  __device__ __forceinline__ void store(float (*xs)[RT + 4]) const {
+#pragma unroll
+    for (int rep = 0; rep < 2; ++rep) {
+      const int v_id = threadIdx.x + rep * kRouterThreads;
+      const int tt = v_id >> 3, kk = (v_id & 7) * 4;
+      xs[kk + 0][tt] = v[rep].x;
+      xs[kk + 1][tt] = v[rep].y;
+      xs[kk + 2][tt] = v[rep].z;
+      xs[kk + 3][tt] = v[rep].w;
+    }
+  }
+};
 
-// part[z][t][e] = sum over this split's k of x[t,k] * w_r[e,k]  (fp32 FFMA)
+struct WChunk {  // 32 experts x 32 k floats = 256 float4, one per thread
+  float4 v;
+  __device__ __forceinline__ void load(const float* w_r, int64_t E, int64_t d,
+                                       int64_t e0, int64_t k0, int64_t kend) {
+    const int64_t e = e0 + (threadIdx.x >> 3), k = k0 + (threadIdx.x & 7) * 4;
+    v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (e < E && k < kend) v = *reinterpret_cast<const float4*>(w_r + e * d + k);
+  }
+  __device__ __forceinline__ void store(float (*wsm)[RE + 4]) const {
+    const int ee = threadIdx.x >> 3, kk = (threadIdx.x & 7) * 4;
+    wsm[kk + 0][ee] = v.x;
+    wsm[kk + 1][ee] = v.y;
+    wsm[kk + 2][ee] = v.z;
+    wsm[kk + 3][ee] = v.w;
+  }
+};
+
+// part[z][t][e] = sum over this split's k of x[t,k] * w_r[e,k]  (fp32 FFMA).
+// The next chunk is loaded into registers while the current one is used.
 template <typename XT>
 __global__ void __launch_bounds__(kRouterThreads)
     router_logits_kernel(const XT* __restrict__ x, const float* __restrict__ w_r,
@@ -88,6 +113,7 @@ __global__ void __launch_bounds__(kRouterThreads)
                          int64_t E, int64_t k_per_split) {
   __shared__ __align__(16) float xs[RK][RT + 4];
   __shared__ __align__(16) float wsm[RK][RE + 4];
+  griddep_wait();
   const int tid = threadIdx.x;
   const int tx = tid & 15;  // expert pair
   const int ty = tid >> 4;  // token quad
@@ -100,22 +126,20 @@ __global__ void __launch_bounds__(kRouterThreads)
 #pragma unroll
   for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = 0.f;
 
+  XChunk<XT> xc;
+  WChunk wc;
+  if (kbeg < kend) {
+    xc.load(x, T, d, t0, kbeg, kend);
+    wc.load(w_r, E, d, e0, kbeg, kend);
+  }
   for (int64_t k0 = kbeg; k0 < kend; k0 += RK) {
-    load_x_chunk<XT>(x, T, d, t0, k0, kend, xs);
-    {  // 32 experts x 32 k floats = 256 float4, one per thread
-      const int ee = tid >> 3;
-      const int kk = (tid & 7) * 4;
-      const int64_t e = e0 + ee;
-      const int64_t k = k0 + kk;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (e < E && k < kend)
-        v = *reinterpret_cast<const float4*>(w_r + e * d + k);
-      wsm[kk + 0][ee] = v.x;
-      wsm[kk + 1][ee] = v.y;
-      wsm[kk + 2][ee] = v.z;
-      wsm[kk + 3][ee] = v.w;
-    }
+    xc.store(xs);
+    wc.store(wsm);
     __syncthreads();
+    if (k0 + RK < kend) {
+      xc.load(x, T, d, t0, k0 + RK, kend);
+      wc.load(w_r, E, d, e0, k0 + RK, kend);
+    }
 #pragma unroll 8
     for (int kk = 0; kk < RK; ++kk) {
       const float4 xv = *reinterpret_cast<const float4*>(&xs[kk][ty * 4]);
@@ -131,6 +155,7 @@ __global__ void __launch_bounds__(kRouterThreads)
     }
     __syncthreads();
   }
+  griddep_launch_dependents();
   float* out = part + (int64_t)blockIdx.z * T * E;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -161,23 +186,33 @@ __global__ void __launch_bounds__(256)
                 const float* __restrict__ bias, float* __restrict__ logits_out,
                 int32_t* __restrict__ idx_out, float* __restrict__ gate_out,
                 uint8_t* __restrict__ flags, int64_t T, int E, int k) {
+  griddep_wait();
   const int lane = threadIdx.x & 31;
   const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  griddep_launch_dependents();
   if (t >= T) return;
 
+  // logits = partial sums added in split order (fixed, so reproducible); the
+  // loads of several splits are issued together
   float lg[PL], key[PL];
+#pragma unroll
+  for (int i = 0; i < PL; ++i) lg[i] = 0.f;
+  const float* pt = part + t * E + lane;
+  const int64_t zstride = T * E;
+#pragma unroll 4
+  for (int z = 0; z < nsplit; ++z) {
+#pragma unroll
+    for (int i = 0; i < PL; ++i)
+      if (lane + 32 * i < E) lg[i] += pt[z * zstride + 32 * i];
+  }
 #pragma unroll
   for (int i = 0; i < PL; ++i) {
     const int e = lane + 32 * i;
-    lg[i] = 0.f;
     key[i] = -INFINITY;
     if (e < E) {
-      float l = 0.f;
-      for (int z = 0; z < nsplit; ++z) l += part[((int64_t)z * T + t) * E + e];
-      lg[i] = l;
-      float kv = l + bias[e];
+      const float kv = lg[i] + bias[e];
       key[i] = (kv != kv) ? -INFINITY : kv;  // a NaN key never wins
-      if (logits_out) logits_out[t * E + e] = l;
+      if (logits_out) logits_out[t * E + e] = lg[i];
     }
   }
 
@@ -247,8 +282,8 @@ void launch_topk(const float* part, int nsplit, const float* bias,
                  int64_t T, int E, int k, cudaStream_t st) {
   const int warps = 8;
   const unsigned grid = (unsigned)((T + warps - 1) / warps);
-  topk_kernel<PL><<<grid, warps * 32, 0, st>>>(part, nsplit, bias, logits, idx,
-                                               gate, flags, T, E, k);
+  launch_pdl(topk_kernel<PL>, dim3(grid), dim3(warps * 32), 0, st, part, nsplit, bias,
+             logits, idx, gate, flags, T, E, k);
 }
 
 }  // namespace
@@ -256,8 +291,9 @@ void launch_topk(const float* part, int nsplit, const float* bias,
 // Number of contraction splits so that the logits GEMM has >= ~2 CTAs per SM.
 int router_splits(const Shape& sh) {
   const int64_t tiles = ((sh.E + RE - 1) / RE) * ((sh.T + RT - 1) / RT);
-  int64_t want = (296 + tiles - 1) / tiles;
-  const int64_t max_split = (sh.d + 255) / 256;  // >= 256 k per split
+  int64_t want = (2 * num_sms() + tiles - 1) / tiles;
+  int64_t max_split = (sh.d + 127) / 128;  // >= 128 k per split
+  if (max_split > 32) max_split = 32;
   if (want > max_split) want = max_split;
   if (want < 1) want = 1;
   return (int)want;
@@ -273,11 +309,11 @@ cudaError_t launch_router(const Shape& sh, const void* x, const float* w_r,
   dim3 grid((unsigned)((sh.E + RE - 1) / RE), (unsigned)((sh.T + RT - 1) / RT),
             (unsigned)nsplit);
   if (sh.bf16)
-    router_logits_kernel<__nv_bfloat16><<<grid, kRouterThreads, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(x), w_r, part, sh.T, sh.d, sh.E, kps);
+    launch_pdl(router_logits_kernel<__nv_bfloat16>, grid, dim3(kRouterThreads), 0, st,
+               static_cast<const __nv_bfloat16*>(x), w_r, part, sh.T, sh.d, sh.E, kps);
   else
-    router_logits_kernel<float><<<grid, kRouterThreads, 0, st>>>(
-        static_cast<const float*>(x), w_r, part, sh.T, sh.d, sh.E, kps);
+    launch_pdl(router_logits_kernel<float>, grid, dim3(kRouterThreads), 0, st,
+               static_cast<const float*>(x), w_r, part, sh.T, sh.d, sh.E, kps);
   const int pl = (int)((sh.E + 31) / 32);
   const int E = (int)sh.E, k = (int)sh.k;
   if (pl <= 1)

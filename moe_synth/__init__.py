@@ -79,6 +79,12 @@ CONFIGS: Dict[str, MoEShape] = {
     # bf16 large-expert-count layer, ~30 % of slots on zero experts
     "large_e": MoEShape("large_e", T=8192, d=6144, n_routed=256, n_zero=64,
                         top_k=12, ffn=2048, routing="zero_share"),
+    # small cases of the same kernels for profiler captures (weights ~0.8 GB,
+    # still larger than L2)
+    "profile_decode": MoEShape("profile_decode", T=64, d=4096, n_routed=32,
+                               n_zero=8, top_k=8, ffn=1024),
+    "profile_prefill": MoEShape("profile_prefill", T=4096, d=4096, n_routed=32,
+                                n_zero=8, top_k=8, ffn=1024, routing="zipf"),
 }
 
 SWEEP_T = (1, 8, 64, 512, 4096, 32768)

@@ -91,14 +91,14 @@ def run_staged_and_fused(sh: MoEShape, seed: int, sample=None, s=None):
         err = rel_rms_err(got, y_ref)
         assert err <= OUT_RTOL_RMS, f"expert rows: max err {err:.3e} x rms"
 
-    # ---- combine, fed the oracle's gates and expert outputs (rounded to act dtype)
+    # ---- combine, fed the oracle's gates and expert outputs (rounded to fp32)
     tok = np.arange(T) if sample is None else np.unique(
         np.random.default_rng(seed + 7).choice(T, size=min(sample, T), replace=False))
     if sample is None and R > 0:
         y_all = oracle.expert_rows(inp.w_gate, inp.w_up, inp.w_down, row_expert,
                                    x_perm_ref[:R])
-        y_in = torch.zeros(T * k, sh.d, dtype=inp.x.dtype)
-        y_in[:R] = torch.from_numpy(y_all).to(inp.x.dtype)
+        y_in = torch.zeros(T * k, sh.d, dtype=torch.float32)
+        y_in[:R] = torch.from_numpy(y_all).float()
         gate32 = torch.from_numpy(ref_gate).float()
         out_c = moe.combine(ls, d_inp.x, y_in.to(DEV), torch.from_numpy(ref_idx).to(DEV),
                             gate32.to(DEV), torch.from_numpy(r_slot_row).to(DEV))
