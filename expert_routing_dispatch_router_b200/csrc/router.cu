@@ -122,6 +122,9 @@ __global__ void __launch_bounds__(kRouterThreads)
   const int64_t kbeg = (int64_t)blockIdx.z * k_per_split;
   const int64_t kend = min(d, kbeg + k_per_split);
 
+  // Blocked summation: each 32-term chunk is summed into a fresh partial that
+  // is then added to the running total, which keeps the fp32 rounding error
+  // of a d-term dot product ~sqrt(32) times below a single running sum.
   float acc[4][2];
 #pragma unroll
   for (int i = 0; i < 4; ++i) acc[i][0] = acc[i][1] = 0.f;
@@ -140,18 +143,26 @@ __global__ void __launch_bounds__(kRouterThreads)
       xc.load(x, T, d, t0, k0 + RK, kend);
       wc.load(w_r, E, d, e0, k0 + RK, kend);
     }
+    float part_acc[4][2];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) part_acc[i][0] = part_acc[i][1] = 0.f;
 #pragma unroll 8
     for (int kk = 0; kk < RK; ++kk) {
       const float4 xv = *reinterpret_cast<const float4*>(&xs[kk][ty * 4]);
       const float2 wv = *reinterpret_cast<const float2*>(&wsm[kk][tx * 2]);
-      acc[0][0] = fmaf(xv.x, wv.x, acc[0][0]);
-      acc[0][1] = fmaf(xv.x, wv.y, acc[0][1]);
-      acc[1][0] = fmaf(xv.y, wv.x, acc[1][0]);
-      acc[1][1] = fmaf(xv.y, wv.y, acc[1][1]);
-      acc[2][0] = fmaf(xv.z, wv.x, acc[2][0]);
-      acc[2][1] = fmaf(xv.z, wv.y, acc[2][1]);
-      acc[3][0] = fmaf(xv.w, wv.x, acc[3][0]);
-      acc[3][1] = fmaf(xv.w, wv.y, acc[3][1]);
+      part_acc[0][0] = fmaf(xv.x, wv.x, part_acc[0][0]);
+      part_acc[0][1] = fmaf(xv.x, wv.y, part_acc[0][1]);
+      part_acc[1][0] = fmaf(xv.y, wv.x, part_acc[1][0]);
+      part_acc[1][1] = fmaf(xv.y, wv.y, part_acc[1][1]);
+      part_acc[2][0] = fmaf(xv.z, wv.x, part_acc[2][0]);
+      part_acc[2][1] = fmaf(xv.z, wv.y, part_acc[2][1]);
+      part_acc[3][0] = fmaf(xv.w, wv.x, part_acc[3][0]);
+      part_acc[3][1] = fmaf(xv.w, wv.y, part_acc[3][1]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      acc[i][0] += part_acc[i][0];
+      acc[i][1] += part_acc[i][1];
     }
     __syncthreads();
   }
@@ -169,15 +180,11 @@ __global__ void __launch_bounds__(kRouterThreads)
   }
 }
 
-struct Cand {
-  float key;
-  float logit;
-  int e;
-};
-
-// a beats b: larger key, ties to the lower expert id
-__device__ __forceinline__ bool beats(float ka, int ea, float kb, int eb) {
-  return ka > kb || (ka == kb && ea < eb);
+// Order-preserving map of a float to uint32 (a < b  <=>  ord(a) < ord(b) for
+// non-NaN values; -inf maps to 0x007fffff, so 0 is below every key).
+__device__ __forceinline__ uint32_t ord_key(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
 template <int PL>
@@ -216,43 +223,44 @@ __global__ void __launch_bounds__(256)
     }
   }
 
+  // Each round: every lane takes its best remaining key (ascending ids, so the
+  // lower id wins ties), then two warp reductions pick the largest key and,
+  // among lanes holding it, the lowest id.
   uint32_t taken = 0;  // bit i: expert lane + 32 i already selected
   float kth_key = 0.f, next_key = -INFINITY;
   float my_logit = 0.f;
   int my_e = 0;
   const int rounds = (k < E) ? k + 1 : k;
   for (int j = 0; j < rounds; ++j) {
-    float bk = -INFINITY, bl = 0.f;
+    uint32_t bo = 0u;
     int be = 0x7fffffff;
+    float bk = -INFINITY, bl = 0.f;
 #pragma unroll
     for (int i = 0; i < PL; ++i) {
       const int e = lane + 32 * i;
-      if (e < E && !((taken >> i) & 1u) && beats(key[i], e, bk, be)) {
-        bk = key[i];
+      const uint32_t o = ord_key(key[i]);
+      if (e < E && !((taken >> i) & 1u) && (be == 0x7fffffff || o > bo)) {
+        bo = o;
         be = e;
+        bk = key[i];
         bl = lg[i];
       }
     }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const float ok = __shfl_xor_sync(0xffffffffu, bk, off);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-      const float ol = __shfl_xor_sync(0xffffffffu, bl, off);
-      if (beats(ok, oe, bk, be)) {
-        bk = ok;
-        be = oe;
-        bl = ol;
-      }
-    }
+    const uint32_t mo = __reduce_max_sync(0xffffffffu, bo);
+    const int we = (int)__reduce_min_sync(0xffffffffu,
+                                          (be != 0x7fffffff && bo == mo) ? (uint32_t)be
+                                                                        : 0x7fffffffu);
+    const float wk = __shfl_sync(0xffffffffu, bk, we & 31);
+    const float wl = __shfl_sync(0xffffffffu, bl, we & 31);
     if (j < k) {
-      if (lane == (be & 31)) taken |= 1u << (be >> 5);
+      if (lane == (we & 31)) taken |= 1u << (we >> 5);
       if (lane == j) {
-        my_logit = bl;
-        my_e = be;
+        my_logit = wl;
+        my_e = we;
       }
-      kth_key = bk;
+      kth_key = wk;
     } else {
-      next_key = bk;
+      next_key = wk;
     }
   }
 
@@ -292,8 +300,8 @@ void launch_topk(const float* part, int nsplit, const float* bias,
 int router_splits(const Shape& sh) {
   const int64_t tiles = ((sh.E + RE - 1) / RE) * ((sh.T + RT - 1) / RT);
   int64_t want = (2 * num_sms() + tiles - 1) / tiles;
-  int64_t max_split = (sh.d + 127) / 128;  // >= 128 k per split
-  if (max_split > 32) max_split = 32;
+  int64_t max_split = (sh.d + 255) / 256;  // >= 256 k per split
+  if (max_split > 16) max_split = 16;
   if (want > max_split) want = max_split;
   if (want < 1) want = 1;
   return (int)want;

@@ -9,8 +9,17 @@ Tolerances (stated for the layer as a whole, derived per stage):
   * gates: |g_gpu - g_ref| <= 2e-5 (a logit error of 1e-5 moves a softmax
     weight by at most ~g * 2e-5)
   * dispatch (counts, offsets, permutation, slot rows, gathered rows): exact
-  * expert rows and layer output: max |gpu - ref| <= 2e-2 * rms(ref)
-    (bf16 inputs, fp32 accumulation, h and y rounded to bf16)
+  * expert rows: max |gpu - ref| <= 2e-2 * rms(ref)  (bf16 inputs, fp32
+    accumulation, h rounded to bf16, y kept in fp32)
+  * layer output: max over elements of (|gpu - ref| - ulp(ref)/2) <= 2e-2 *
+    rms(ref), where ulp is the spacing of the output format (bf16: 8
+    significant bits) at ref. The 2e-2 * rms bound covers the arithmetic; the
+    output is then stored in the activation format, which by itself moves an
+    element by up to half an ulp. Without that term no implementation with a
+    bf16 output could pass: the exact fp64 result rounded to bf16 already
+    differs from itself by 2.6e-2 to 2.9e-2 x rms on the decode workload,
+    whose outputs reach 8-10 x rms (test_tolerance_reading.py shows the
+    effect on a constructed case).
 """
 import numpy as np
 import torch
@@ -26,6 +35,24 @@ def rel_rms_err(got, ref):
     ref = np.asarray(ref, dtype=np.float64)
     rms = float(np.sqrt(np.mean(ref * ref)))
     return float(np.max(np.abs(got - ref))) / max(rms, 1e-30)
+
+
+def half_ulp(ref, dtype):
+    """Half the spacing of the output format at |ref| (bf16: p = 8 bits,
+    fp32: p = 24 bits): 2^(floor(log2|ref|) - p)."""
+    p = {torch.bfloat16: 8, torch.float32: 24}[dtype]
+    a = np.maximum(np.abs(np.asarray(ref, dtype=np.float64)), 1e-300)
+    return np.exp2(np.floor(np.log2(a)) - p)
+
+
+def out_err(got, ref, dtype):
+    """max(|got - ref| - ulp(ref)/2) / rms(ref): the arithmetic error of a
+    result stored in `dtype`, relative to the reference's RMS."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    rms = float(np.sqrt(np.mean(ref * ref)))
+    excess = np.abs(got - ref) - half_ulp(ref, dtype)
+    return float(np.max(excess, initial=0.0)) / max(rms, 1e-30)
 
 
 def assert_logits_close(gpu_logits, ref_logits):
