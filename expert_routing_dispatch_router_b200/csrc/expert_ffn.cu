@@ -43,19 +43,16 @@ namespace moe {
 namespace {
 
 // ------------------------------------------------------------------ plan --
-// tile_start[e] = sum over routed e' < e of ceil(count[e'] / kTileTokens);
-// tile_start[N] = total token tiles. One block; N <= 1024.
-__global__ void __launch_bounds__(1024)
-    gemm_plan_kernel(const int32_t* __restrict__ offsets, int N,
-                     int32_t* __restrict__ tile_start) {
-  __shared__ int32_t warp_sums[32];
-  griddep_wait();
-  griddep_launch_dependents();
+// For token tiles of `tile` rows: tile_start[e] = sum over routed e' < e of
+// ceil(count[e'] / tile); tile_start[N] = total token tiles. One block; N <= 1024.
+__device__ __forceinline__ void tile_prefix(const int32_t* __restrict__ offsets, int N,
+                                            int tile, int32_t* __restrict__ tile_start,
+                                            int32_t* warp_sums) {
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   int32_t v = 0;
   if ((int)threadIdx.x < N) {
     const int32_t n = offsets[threadIdx.x + 1] - offsets[threadIdx.x];
-    v = (n + kTileTokens - 1) / kTileTokens;
+    v = (n + tile - 1) / tile;
   }
   int32_t incl = v;
 #pragma unroll
@@ -78,23 +75,41 @@ __global__ void __launch_bounds__(1024)
   const int32_t before = (wid > 0 ? warp_sums[wid - 1] : 0) + incl - v;
   if ((int)threadIdx.x < N) tile_start[threadIdx.x] = before;
   if (threadIdx.x == 0) tile_start[N] = warp_sums[31];
+  __syncthreads();
+}
+
+// Plans of both expert GEMMs: gate/up tiles of kTileGateUp tokens into
+// tile_start[0..N], down tiles of kTileDown tokens into tile_start[N+1..2N+1].
+__global__ void __launch_bounds__(1024)
+    gemm_plan_kernel(const int32_t* __restrict__ offsets, int N,
+                     int32_t* __restrict__ tile_start) {
+  __shared__ int32_t warp_sums[32];
+  griddep_wait();
+  griddep_launch_dependents();
+  tile_prefix(offsets, N, kTileGateUp, tile_start, warp_sums);
+  tile_prefix(offsets, N, kTileDown, tile_start + N + 1, warp_sums);
 }
 
 // ------------------------------------------------------- tensor-core path --
 constexpr int BM = 128;  // weight rows per tile (MMA M)
 constexpr int BK = 64;   // contraction elements per stage: 128-byte rows
-constexpr int BN = kTileTokens;  // token rows per tile (MMA N, max)
 constexpr int kThreads = 192;
 constexpr uint32_t kTileBytes = BM * BK * 2;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccStride = 256;  // TMEM columns per accumulator buffer
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
+// Gate/up: two weight tiles (W_gate, W_up rows) x 128 tokens, two fp32
+// accumulators of 128 columns. Down: one weight tile x 256 tokens, one
+// accumulator of 256 columns. Either way a TMEM buffer is 256 columns and
+// there are two of them.
 template <bool GATEUP>
 struct Cfg {
   static constexpr int kNumA = GATEUP ? 2 : 1;
-  static constexpr int kStages = GATEUP ? 4 : 6;
-  static constexpr uint32_t kStageBytes = (kNumA + 1) * kTileBytes;
+  static constexpr int BN = GATEUP ? kTileGateUp : kTileDown;  // max MMA N
+  static constexpr uint32_t kBBytes = BN * BK * 2;
+  static constexpr uint32_t kStageBytes = kNumA * kTileBytes + kBBytes;
+  static constexpr int kStages = (GATEUP ? 4 : 4);
   static constexpr uint32_t kBarOff = kStages * kStageBytes;
   static constexpr uint32_t kTabOff = kBarOff + 256;
   static constexpr uint32_t kSmemBytes =
@@ -113,9 +128,10 @@ struct GemmArgs {
 };
 
 struct Unit {
-  int e, m, row0, n_valid, n_mma;
+  int e, m, row0, n_valid, n_mma, ntiles;
 };
 
+template <int BN>
 __device__ __forceinline__ Unit decode_unit(int u, const int* s_tiles,
                                             const int* s_offs, int N,
                                             int m_tiles) {
@@ -130,6 +146,7 @@ __device__ __forceinline__ Unit decode_unit(int u, const int* s_tiles,
   Unit un;
   un.e = lo;
   const int ntiles = s_tiles[lo + 1] - s_tiles[lo];
+  un.ntiles = ntiles;
   const int local = u - m_tiles * s_tiles[lo];
   un.m = local / ntiles;
   const int tt = local - un.m * ntiles;
@@ -178,6 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                            const GemmArgs args) {
   using C = Cfg<GATEUP>;
   constexpr int S = C::kStages;
+  constexpr int BN = C::BN;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -235,15 +253,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ---------------------------------------------------- TMA producer --
     if (lane == 0) {
-      const uint64_t pol_w = ptx::policy_evict_first();
-      const uint64_t pol_x = ptx::policy_evict_last();
+      // L2 policy per unit: an expert with a single token tile reads each
+      // weight tile once (a decode step), so its weights are streamed
+      // evict-first and its few token rows kept evict-last. An expert with
+      // several token tiles reuses every weight tile once per token tile, so
+      // both operands use the normal policy.
+      const uint64_t pol_first = ptx::policy_evict_first();
+      const uint64_t pol_last = ptx::policy_evict_last();
+      const uint64_t pol_normal = ptx::policy_evict_normal();
       int stage = 0;
       uint32_t phase = 0, armed = 0, armed_par = 0;
       bool ok = true;
       for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
-        const Unit un = decode_unit(u, s_tiles, s_offs, N, args.m_tiles);
+        const Unit un = decode_unit<BN>(u, s_tiles, s_offs, N, args.m_tiles);
         const int arow = un.e * args.out_cols + un.m * BM;
         const uint32_t bytes = C::kNumA * kTileBytes + (uint32_t)un.n_mma * 128u;
+        const uint64_t pol_w = un.ntiles == 1 ? pol_first : pol_normal;
+        const uint64_t pol_x = un.ntiles == 1 ? pol_last : pol_normal;
         for (int kb = 0; kb < args.num_kb; ++kb) {
           if (!wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, args.err)) {
             ok = false;
@@ -254,14 +280,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t a0 = sbase + stage * C::kStageBytes;
           ptx::tma_load_2d(&tmA0, a0, fb, kb * BK, arow, pol_w);
           if (GATEUP) ptx::tma_load_2d(&tmA1, a0 + kTileBytes, fb, kb * BK, arow, pol_w);
+          // token rows: 128-row boxes while 128 or more remain, then 16-row boxes
           const uint32_t b0 = a0 + C::kNumA * kTileBytes;
-          if (un.n_mma == BN) {
-            ptx::tma_load_2d(&tmB128, b0, fb, kb * BK, un.row0, pol_x);
-          } else {
-            for (int j = 0; j < un.n_mma / 16; ++j)
-              ptx::tma_load_2d(&tmB16, b0 + j * 2048u, fb, kb * BK, un.row0 + 16 * j,
-                               pol_x);
-          }
+          int j = 0;
+          for (; j + 128 <= un.n_mma; j += 128)
+            ptx::tma_load_2d(&tmB128, b0 + j * 128u, fb, kb * BK, un.row0 + j, pol_x);
+          for (; j < un.n_mma; j += 16)
+            ptx::tma_load_2d(&tmB16, b0 + j * 128u, fb, kb * BK, un.row0 + j, pol_x);
           armed |= 1u << stage;
           armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
           if (++stage == S) {
@@ -282,7 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true, issued = false;
       for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
-        const Unit un = decode_unit(u, s_tiles, s_offs, N, args.m_tiles);
+        const Unit un = decode_unit<BN>(u, s_tiles, s_offs, N, args.m_tiles);
         if (!wait_bounded(tempty_bar(acc), acc_phase ^ 1u, abort_flag, args.err)) {
           ok = false;
           break;
@@ -331,7 +356,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int u = blockIdx.x; u < total_units; u += gridDim.x) {
-      const Unit un = decode_unit(u, s_tiles, s_offs, N, args.m_tiles);
+      const Unit un = decode_unit<BN>(u, s_tiles, s_offs, N, args.m_tiles);
       const bool ok = wait_bounded(tfull_bar(acc), acc_phase, abort_flag, args.err);
       if (!__all_sync(0xffffffffu, ok)) break;
       ptx::tc_fence_after();
@@ -510,6 +535,30 @@ cudaError_t launch_simt(const Shape& sh, const void* x_perm, const int32_t* offs
 
 }  // namespace
 
+// out[T, M] (fp32) = b[T, K] (bf16) * a[M, K]^T (bf16) on the tensor cores, run
+// as one "expert" of the grouped kernel's down variant. M is a multiple of 128
+// and K of 64. plan is a device int32[4] holding {0, T, 0, ceil(T / kTileDown)}
+// (that expert's row offsets, then its token-tile prefix).
+cudaError_t launch_dense_gemm_tc(const void* a, int64_t M, const void* b, int64_t T,
+                                 int64_t K, float* out, const int32_t* plan,
+                                 int32_t* err, cudaStream_t st) {
+  CUtensorMap am, b16, b128;
+  if (!make_map(&am, a, (uint64_t)M, (uint64_t)K, BM) ||
+      !make_map(&b16, b, (uint64_t)T, (uint64_t)K, 16) ||
+      !make_map(&b128, b, (uint64_t)T, (uint64_t)K, 128))
+    return cudaErrorInvalidValue;
+  GemmArgs g;
+  g.offsets = plan;
+  g.tile_start = plan + 2;
+  g.out = out;
+  g.err = err;
+  g.N = 1;
+  g.num_kb = (int)(K / BK);
+  g.out_cols = (int)M;
+  g.m_tiles = (int)(M / BM);
+  return launch_tc<false>(am, am, b16, b128, g, st);
+}
+
 bool expert_ffn_uses_tensor_cores(const Shape& sh) {
   return sh.bf16 && sh.d % 128 == 0 && sh.F % 128 == 0 && sh.N <= kMaxExperts;
 }
@@ -538,9 +587,9 @@ cudaError_t launch_expert_ffn(const Shape& sh, const void* x_perm,
       make_map(&wu_map, w_up, (uint64_t)(sh.N * sh.F), (uint64_t)sh.d, BM) &&
       make_map(&wd_map, w_down, (uint64_t)(sh.N * sh.d), (uint64_t)sh.F, BM) &&
       make_map(&x16, x_perm, rows_cap, (uint64_t)sh.d, 16) &&
-      make_map(&x128, x_perm, rows_cap, (uint64_t)sh.d, BN) &&
+      make_map(&x128, x_perm, rows_cap, (uint64_t)sh.d, 128) &&
       make_map(&h16, h, rows_cap, (uint64_t)sh.F, 16) &&
-      make_map(&h128, h, rows_cap, (uint64_t)sh.F, BN);
+      make_map(&h128, h, rows_cap, (uint64_t)sh.F, 128);
   if (!ok) return cudaErrorInvalidValue;
 
   cudaError_t e = launch_pdl(gemm_plan_kernel, dim3(1), dim3(1024), 0, st, offsets,
@@ -560,6 +609,7 @@ cudaError_t launch_expert_ffn(const Shape& sh, const void* x_perm,
   if (e != cudaSuccess) return e;
 
   GemmArgs dn = gu;
+  dn.tile_start = tile_start + sh.N + 1;
   dn.out = y_perm;
   dn.num_kb = (int)(sh.F / BK);
   dn.out_cols = (int)sh.d;

@@ -23,7 +23,14 @@ WsLayout ws_layout(const Shape& sh) {
   };
   const size_t Tk = (size_t)(sh.T * sh.k);
   L.header = take(256);
-  L.logits = take((size_t)router_splits(sh) * sh.T * sh.E * sizeof(float));
+  size_t part = (size_t)router_splits(sh) * sh.T * sh.E;
+  const size_t tc_part = (size_t)sh.T * router_planes_rows(sh);
+  if (router_uses_tensor_cores(sh) && tc_part > part) part = tc_part;
+  L.logits = take(part * sizeof(float));
+  L.planes = take(router_uses_tensor_cores(sh)
+                      ? (size_t)router_planes_rows(sh) * sh.d * sizeof(uint16_t)
+                      : 0);
+  L.router_plan = take(4 * sizeof(int32_t));
   L.topk_idx = take(Tk * sizeof(int32_t));
   L.topk_gate = take(Tk * sizeof(float));
   L.chunk_base = take((size_t)sh.nchunks * sh.E * sizeof(int32_t));
@@ -31,7 +38,7 @@ WsLayout ws_layout(const Shape& sh) {
   L.offsets = take((size_t)(sh.N + 1) * sizeof(int32_t));
   L.row_token = take(Tk * sizeof(int32_t));
   L.slot_row = take(Tk * sizeof(int32_t));
-  L.tile_start = take((size_t)(sh.N + 1) * sizeof(int32_t));
+  L.tile_start = take(2 * (size_t)(sh.N + 1) * sizeof(int32_t));
   L.x_perm = take(Tk * sh.d * sh.es);
   L.h = take(Tk * sh.F * sh.es);
   L.y_perm = take(Tk * sh.d * sizeof(float));
@@ -107,7 +114,8 @@ moe_status_t run_layer(const Shape& sh, const void* x, const float* w_router,
   void* x_perm = at<void>(ws, L.x_perm);
   void* y_perm = at<void>(ws, L.y_perm);
   cudaError_t e = launch_router(sh, x, w_router, bias, at<float>(ws, L.logits), idx,
-                                gate, nullptr, nullptr, st);
+                                gate, nullptr, nullptr, at<void>(ws, L.planes),
+                                at<int32_t>(ws, L.router_plan), err, st);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   e = launch_dispatch(sh, x, idx, at<int32_t>(ws, L.chunk_base),
                       counts ? counts : at<int32_t>(ws, L.counts), offsets,
@@ -145,6 +153,8 @@ moe_status_t moe_route(const moe_config_t* cfg, const void* x, const float* w_ro
   const WsLayout L = ws_layout(sh);
   return cuda_status(launch_router(sh, x, w_router, bias, at<float>(ws, L.logits),
                                    topk_idx, topk_gate, flags, logits,
+                                   at<void>(ws, L.planes), at<int32_t>(ws, L.router_plan),
+                                   at<int32_t>(ws, L.header),
                                    reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -274,7 +284,7 @@ moe_status_t moe_read_device_error(void* ws, int32_t* code_out, moe_stream_t str
 int32_t moe_layer_launch_count(const moe_config_t* cfg) {
   Shape sh;
   if (make_shape(cfg, &sh) != MOE_OK || sh.T == 0) return 0;
-  int32_t n = 2;                  // router logits + top-k
+  int32_t n = router_launch_count(sh);  // (split + GEMM | logits) + top-k
   n += dispatch_launch_count(sh);  // (count, scan, scatter | small) + gather
   n += expert_ffn_launch_count(sh);
   n += 1;                         // combine

@@ -15,7 +15,8 @@ namespace moe {
 constexpr int kMaxExperts = 1024;  // top-k keeps E/32 keys per lane
 constexpr int kMaxTopK = 32;       // one gate per lane
 constexpr int kChunkTokens = 256;  // tokens per dispatch block
-constexpr int kTileTokens = 128;   // token tile of the expert GEMMs
+constexpr int kTileGateUp = 128;   // token tile of the gate/up expert GEMM
+constexpr int kTileDown = 256;     // token tile of the down expert GEMM
 constexpr int kWsAlign = 1024;
 
 // Device error codes written into the workspace header.
@@ -26,7 +27,9 @@ constexpr int kErrBadExpertId = 2;
 // from the config alone; every region is kWsAlign-aligned.
 struct WsLayout {
   size_t header;       // int32[64]: [0] error code, [1] error detail
-  size_t logits;       // float [splits, T, E] router partial sums
+  size_t logits;       // float router partials: [splits, T, E] or [T, 3E pad]
+  size_t planes;       // bf16 [3E pad, d] router weights split in 3 planes
+  size_t router_plan;  // int32 [4] plan of the tensor-core router GEMM
   size_t topk_idx;     // int32 [T, k]
   size_t topk_gate;    // float [T, k]
   size_t chunk_base;   // int32 [nchunks, E]
@@ -34,7 +37,7 @@ struct WsLayout {
   size_t offsets;      // int32 [N + 1]
   size_t row_token;    // int32 [T*k]
   size_t slot_row;     // int32 [T*k]
-  size_t tile_start;   // int32 [N + 1] (expert GEMM plan)
+  size_t tile_start;   // int32 [2 (N + 1)] (expert GEMM plans)
   size_t x_perm;       // act   [T*k, d]
   size_t h;            // act   [T*k, F]
   size_t y_perm;       // float [T*k, d]
@@ -58,6 +61,7 @@ int router_splits(const Shape& sh);
 cudaError_t launch_router(const Shape& sh, const void* x, const float* w_r,
                           const float* bias, float* part, int32_t* idx,
                           float* gate, uint8_t* flags, float* logits_out,
+                          void* planes, int32_t* plan, int32_t* err,
                           cudaStream_t st);
 cudaError_t launch_dispatch(const Shape& sh, const void* x, const int32_t* idx,
                             int32_t* chunk_base, int32_t* counts,
@@ -72,6 +76,12 @@ cudaError_t launch_expert_ffn(const Shape& sh, const void* x_perm,
 cudaError_t launch_combine(const Shape& sh, const void* x, const void* y_perm,
                            const int32_t* idx, const float* gate,
                            const int32_t* slot_row, void* out, cudaStream_t st);
+cudaError_t launch_dense_gemm_tc(const void* a, int64_t M, const void* b, int64_t T,
+                                 int64_t K, float* out, const int32_t* plan,
+                                 int32_t* err, cudaStream_t st);
+bool router_uses_tensor_cores(const Shape& sh);
+int64_t router_planes_rows(const Shape& sh);   // 3E rounded up to 128
+int router_launch_count(const Shape& sh);
 int expert_ffn_launch_count(const Shape& sh);
 int dispatch_launch_count(const Shape& sh);
 bool expert_ffn_uses_tensor_cores(const Shape& sh);

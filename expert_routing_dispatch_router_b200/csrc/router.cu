@@ -189,7 +189,8 @@ __device__ __forceinline__ uint32_t ord_key(float f) {
 
 template <int PL>
 __global__ void __launch_bounds__(256)
-    topk_kernel(const float* __restrict__ part, int nsplit,
+    topk_kernel(const float* __restrict__ part, int nsplit, int64_t row_stride,
+                int64_t split_stride,
                 const float* __restrict__ bias, float* __restrict__ logits_out,
                 int32_t* __restrict__ idx_out, float* __restrict__ gate_out,
                 uint8_t* __restrict__ flags, int64_t T, int E, int k) {
@@ -204,8 +205,8 @@ __global__ void __launch_bounds__(256)
   float lg[PL], key[PL];
 #pragma unroll
   for (int i = 0; i < PL; ++i) lg[i] = 0.f;
-  const float* pt = part + t * E + lane;
-  const int64_t zstride = T * E;
+  const float* pt = part + t * row_stride + lane;
+  const int64_t zstride = split_stride;
 #pragma unroll 4
   for (int z = 0; z < nsplit; ++z) {
 #pragma unroll
@@ -285,16 +286,81 @@ __global__ void __launch_bounds__(256)
 }
 
 template <int PL>
-void launch_topk(const float* part, int nsplit, const float* bias,
+void launch_topk(const float* part, int nsplit, int64_t row_stride,
+                 int64_t split_stride, const float* bias,
                  float* logits, int32_t* idx, float* gate, uint8_t* flags,
                  int64_t T, int E, int k, cudaStream_t st) {
   const int warps = 8;
   const unsigned grid = (unsigned)((T + warps - 1) / warps);
-  launch_pdl(topk_kernel<PL>, dim3(grid), dim3(warps * 32), 0, st, part, nsplit, bias,
+  launch_pdl(topk_kernel<PL>, dim3(grid), dim3(warps * 32), 0, st, part, nsplit,
+             row_stride, split_stride, bias,
              logits, idx, gate, flags, T, E, k);
 }
 
+// Exact three-way split of the fp32 router weights into bf16 planes for the
+// tensor-core router: hi = bf16(w), mid = bf16(w - hi), lo = bf16(w - hi - mid)
+// (each difference is exact in fp32), so hi + mid + lo carries the 24 bits of
+// w and x . w = x . hi + x . mid + x . lo with x in bf16 and every product
+// exact in fp32. Rows [0,E) of `planes` get hi, [E,2E) mid, [2E,3E) lo, the
+// padding rows up to Ep zeros. Also writes the one-expert plan of the GEMM.
+__global__ void __launch_bounds__(256)
+    router_split_kernel(const float4* __restrict__ w_r, int64_t E, int64_t d, int64_t Ep,
+                        uint2* __restrict__ planes, int32_t* __restrict__ plan,
+                        int64_t T, int tile) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const int64_t q = d / 4;  // float4 per row
+  const int64_t n = E * q;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
+    const float4 w = w_r[i];
+    const float v[4] = {w.x, w.y, w.z, w.w};
+    uint16_t hb[4], mb[4], lb[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const __nv_bfloat16 h = __float2bfloat16_rn(v[j]);
+      const float r1 = v[j] - __bfloat162float(h);
+      const __nv_bfloat16 m = __float2bfloat16_rn(r1);
+      const float r2 = r1 - __bfloat162float(m);
+      const __nv_bfloat16 l = __float2bfloat16_rn(r2);
+      hb[j] = __bfloat16_as_ushort(h);
+      mb[j] = __bfloat16_as_ushort(m);
+      lb[j] = __bfloat16_as_ushort(l);
+    }
+    auto pack = [](const uint16_t* b) {
+      return make_uint2((uint32_t)b[0] | ((uint32_t)b[1] << 16),
+                        (uint32_t)b[2] | ((uint32_t)b[3] << 16));
+    };
+    planes[i] = pack(hb);
+    planes[n + i] = pack(mb);
+    planes[2 * n + i] = pack(lb);
+  }
+  for (int64_t i = 3 * n + (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < Ep * q;
+       i += stride)
+    planes[i] = make_uint2(0u, 0u);
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    plan[0] = 0;
+    plan[1] = (int32_t)T;
+    plan[2] = 0;
+    plan[3] = (int32_t)((T + tile - 1) / tile);
+  }
+}
+
 }  // namespace
+
+// The router runs on the tensor cores (three bf16 planes, fp32 accumulation)
+// for bf16 batches large enough to fill the GPU; small batches and fp32
+// activations use the CUDA-core split-K kernel.
+constexpr int64_t kTcRouterMinTokens = 512;
+
+int64_t router_planes_rows(const Shape& sh) { return (3 * sh.E + 127) / 128 * 128; }
+
+bool router_uses_tensor_cores(const Shape& sh) {
+  return sh.bf16 && sh.d % 128 == 0 && sh.T >= kTcRouterMinTokens &&
+         router_planes_rows(sh) <= 4096;
+}
+
+int router_launch_count(const Shape& sh) { return router_uses_tensor_cores(sh) ? 3 : 2; }
 
 // Number of contraction splits so that the logits GEMM has >= ~2 CTAs per SM.
 int router_splits(const Shape& sh) {
@@ -310,32 +376,60 @@ int router_splits(const Shape& sh) {
 cudaError_t launch_router(const Shape& sh, const void* x, const float* w_r,
                           const float* bias, float* part, int32_t* idx,
                           float* gate, uint8_t* flags, float* logits_out,
+                          void* planes, int32_t* plan, int32_t* err,
                           cudaStream_t st) {
-  const int nsplit = router_splits(sh);
-  int64_t kps = (sh.d + nsplit - 1) / nsplit;
-  kps = (kps + RK - 1) / RK * RK;
-  dim3 grid((unsigned)((sh.E + RE - 1) / RE), (unsigned)((sh.T + RT - 1) / RT),
-            (unsigned)nsplit);
-  if (sh.bf16)
-    launch_pdl(router_logits_kernel<__nv_bfloat16>, grid, dim3(kRouterThreads), 0, st,
-               static_cast<const __nv_bfloat16*>(x), w_r, part, sh.T, sh.d, sh.E, kps);
-  else
-    launch_pdl(router_logits_kernel<float>, grid, dim3(kRouterThreads), 0, st,
-               static_cast<const float*>(x), w_r, part, sh.T, sh.d, sh.E, kps);
+  int nsplit;
+  int64_t row_stride, split_stride;
+  cudaError_t e;
+  if (router_uses_tensor_cores(sh)) {
+    const int64_t Ep = router_planes_rows(sh);
+    const int64_t n4 = sh.E * sh.d / 4;
+    int64_t blocks = (n4 + 255) / 256;
+    if (blocks > 4 * num_sms()) blocks = 4 * num_sms();
+    e = launch_pdl(router_split_kernel, dim3((unsigned)blocks), dim3(256), 0, st,
+                   reinterpret_cast<const float4*>(w_r), sh.E, sh.d, Ep,
+                   static_cast<uint2*>(planes), plan, sh.T, kTileDown);
+    if (e != cudaSuccess) return e;
+    e = launch_dense_gemm_tc(planes, Ep, x, sh.T, sh.d, part, plan, err, st);
+    if (e != cudaSuccess) return e;
+    nsplit = 3;
+    row_stride = Ep;
+    split_stride = sh.E;
+  } else {
+    nsplit = router_splits(sh);
+    int64_t kps = (sh.d + nsplit - 1) / nsplit;
+    kps = (kps + RK - 1) / RK * RK;
+    dim3 grid((unsigned)((sh.E + RE - 1) / RE), (unsigned)((sh.T + RT - 1) / RT),
+              (unsigned)nsplit);
+    if (sh.bf16)
+      e = launch_pdl(router_logits_kernel<__nv_bfloat16>, grid, dim3(kRouterThreads), 0, st,
+                     static_cast<const __nv_bfloat16*>(x), w_r, part, sh.T, sh.d, sh.E,
+                     kps);
+    else
+      e = launch_pdl(router_logits_kernel<float>, grid, dim3(kRouterThreads), 0, st,
+                     static_cast<const float*>(x), w_r, part, sh.T, sh.d, sh.E, kps);
+    if (e != cudaSuccess) return e;
+    row_stride = sh.E;
+    split_stride = sh.T * sh.E;
+  }
   const int pl = (int)((sh.E + 31) / 32);
   const int E = (int)sh.E, k = (int)sh.k;
+#define MOE_TOPK(P)                                                                    \
+  launch_topk<P>(part, nsplit, row_stride, split_stride, bias, logits_out, idx, gate, \
+                 flags, sh.T, E, k, st)
   if (pl <= 1)
-    launch_topk<1>(part, nsplit, bias, logits_out, idx, gate, flags, sh.T, E, k, st);
+    MOE_TOPK(1);
   else if (pl <= 2)
-    launch_topk<2>(part, nsplit, bias, logits_out, idx, gate, flags, sh.T, E, k, st);
+    MOE_TOPK(2);
   else if (pl <= 4)
-    launch_topk<4>(part, nsplit, bias, logits_out, idx, gate, flags, sh.T, E, k, st);
+    MOE_TOPK(4);
   else if (pl <= 8)
-    launch_topk<8>(part, nsplit, bias, logits_out, idx, gate, flags, sh.T, E, k, st);
+    MOE_TOPK(8);
   else if (pl <= 16)
-    launch_topk<16>(part, nsplit, bias, logits_out, idx, gate, flags, sh.T, E, k, st);
+    MOE_TOPK(16);
   else
-    launch_topk<32>(part, nsplit, bias, logits_out, idx, gate, flags, sh.T, E, k, st);
+    MOE_TOPK(32);
+#undef MOE_TOPK
   return cudaGetLastError();
 }
 

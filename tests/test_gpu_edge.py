@@ -161,7 +161,7 @@ def test_router_exact_ties_go_to_lower_id():
     sh = MoEShape("ties", T=96, d=256, n_routed=12, n_zero=4, top_k=6, ffn=128)
     inp = make_inputs(sh, 14, with_experts=False)
     inp.w_router[3:13] = inp.w_router[3]
-    inp.bias[3:13] = 2.0  # the tied group is always selected first
+    inp.bias[3:13] = 50.0  # the tied group is always selected first
     ls = shape_of(sh)
     d = inp.to(DEV)
     ws = moe.alloc_workspace(ls)
