@@ -78,16 +78,16 @@ __device__ __forceinline__ void tile_prefix(const int32_t* __restrict__ offsets,
   __syncthreads();
 }
 
-// Plans of both expert GEMMs: gate/up tiles of kTileGateUp tokens into
-// tile_start[0..N], down tiles of kTileDown tokens into tile_start[N+1..2N+1].
+// Plans of both expert GEMMs: gate/up tiles of tile_gu tokens into
+// tile_start[0..N], down tiles of tile_dn tokens into tile_start[N+1..2N+1].
 __global__ void __launch_bounds__(1024)
-    gemm_plan_kernel(const int32_t* __restrict__ offsets, int N,
+    gemm_plan_kernel(const int32_t* __restrict__ offsets, int N, int tile_gu, int tile_dn,
                      int32_t* __restrict__ tile_start) {
   __shared__ int32_t warp_sums[32];
   griddep_wait();
   griddep_launch_dependents();
-  tile_prefix(offsets, N, kTileGateUp, tile_start, warp_sums);
-  tile_prefix(offsets, N, kTileDown, tile_start + N + 1, warp_sums);
+  tile_prefix(offsets, N, tile_gu, tile_start, warp_sums);
+  tile_prefix(offsets, N, tile_dn, tile_start + N + 1, warp_sums);
 }
 
 // ------------------------------------------------------- tensor-core path --
@@ -99,17 +99,21 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccStride = 256;  // TMEM columns per accumulator buffer
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
-// Gate/up: two weight tiles (W_gate, W_up rows) x 128 tokens, two fp32
-// accumulators of 128 columns. Down: one weight tile x 256 tokens, one
-// accumulator of 256 columns. Either way a TMEM buffer is 256 columns and
-// there are two of them.
-template <bool GATEUP>
+// Gate/up: two weight tiles (W_gate, W_up rows) x up to 128 tokens, two fp32
+// accumulators of <= 128 columns. Down: one weight tile x up to 256 tokens,
+// one accumulator of <= 256 columns. Either way a TMEM buffer is 256 columns
+// and there are two of them. Token tiles are sized to the batch on the host
+// (an expert sees at most T rows): small tiles leave room for more stages, so
+// a decode step keeps more weight bytes in flight.
+template <bool GATEUP, int BN_>
 struct Cfg {
   static constexpr int kNumA = GATEUP ? 2 : 1;
-  static constexpr int BN = GATEUP ? kTileGateUp : kTileDown;  // max MMA N
+  static constexpr int BN = BN_;  // max MMA N
+  static_assert(BN % 16 == 0 && BN <= (GATEUP ? 128 : 256), "token tile");
   static constexpr uint32_t kBBytes = BN * BK * 2;
   static constexpr uint32_t kStageBytes = kNumA * kTileBytes + kBBytes;
-  static constexpr int kStages = (GATEUP ? 4 : 4);
+  static constexpr int kStages =
+      (204800 / kStageBytes) > 8 ? 8 : (int)(204800 / kStageBytes);
   static constexpr uint32_t kBarOff = kStages * kStageBytes;
   static constexpr uint32_t kTabOff = kBarOff + 256;
   static constexpr uint32_t kSmemBytes =
@@ -123,8 +127,11 @@ struct GemmArgs {
   int32_t* err;               // workspace error word
   int N;
   int num_kb;    // contraction length / BK
-  int out_cols;  // F for gate/up, d for down
+  int out_cols;  // output row stride: F for gate/up, d for down
   int m_tiles;   // out_cols / BM
+  int a_rows;    // rows of A per expert (A row = e * a_rows + (m % mt_chunk) * BM)
+  int mt_chunk;  // m-tiles per contraction chunk: m-tile m covers k-blocks
+  int kb_chunk;  // [(m / mt_chunk) * kb_chunk, +kb_chunk) with a fresh accumulator
 };
 
 struct Unit {
@@ -186,14 +193,14 @@ __device__ __forceinline__ void wait_cleanup(uint32_t bar, uint32_t parity) {
 
 __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + __expf(-z)); }
 
-template <bool GATEUP>
+template <bool GATEUP, int BN_>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0,
                            const __grid_constant__ CUtensorMap tmA1,
                            const __grid_constant__ CUtensorMap tmB16,
                            const __grid_constant__ CUtensorMap tmB128,
                            const GemmArgs args) {
-  using C = Cfg<GATEUP>;
+  using C = Cfg<GATEUP, BN_>;
   constexpr int S = C::kStages;
   constexpr int BN = C::BN;
   extern __shared__ uint8_t smem_raw[];
@@ -266,11 +273,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
         const Unit un = decode_unit<BN>(u, s_tiles, s_offs, N, args.m_tiles);
-        const int arow = un.e * args.out_cols + un.m * BM;
+        const int arow = un.e * args.a_rows + (un.m % args.mt_chunk) * BM;
+        const int kb0 = (un.m / args.mt_chunk) * args.kb_chunk;
         const uint32_t bytes = C::kNumA * kTileBytes + (uint32_t)un.n_mma * 128u;
         const uint64_t pol_w = un.ntiles == 1 ? pol_first : pol_normal;
         const uint64_t pol_x = un.ntiles == 1 ? pol_last : pol_normal;
-        for (int kb = 0; kb < args.num_kb; ++kb) {
+        for (int kb = kb0; kb < kb0 + args.kb_chunk; ++kb) {
           if (!wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, args.err)) {
             ok = false;
             break;
@@ -315,7 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::tc_fence_after();
         const uint32_t idesc = ptx::idesc_bf16_f32(BM, un.n_mma);
         const uint32_t d0 = tmem_base + (uint32_t)acc * kAccStride;
-        for (int kb = 0; kb < args.num_kb; ++kb) {
+        for (int kb = 0; kb < args.kb_chunk; ++kb) {
           if (!wait_bounded(full_bar(stage), phase, abort_flag, args.err)) {
             ok = false;
             break;
@@ -427,22 +435,27 @@ bool make_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool GATEUP>
+template <bool GATEUP, int BN>
 cudaError_t launch_tc(const CUtensorMap& a0, const CUtensorMap& a1,
                       const CUtensorMap& b16, const CUtensorMap& b128,
                       const GemmArgs& args, cudaStream_t st) {
-  using C = Cfg<GATEUP>;
+  using C = Cfg<GATEUP, BN>;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_tc_kernel<GATEUP>,
+    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_tc_kernel<GATEUP, BN>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)C::kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  return launch_pdl(grouped_gemm_tc_kernel<GATEUP>, dim3(num_sms()), dim3(kThreads),
+  return launch_pdl(grouped_gemm_tc_kernel<GATEUP, BN>, dim3(num_sms()), dim3(kThreads),
                     C::kSmemBytes, st, a0, a1, b16, b128, args);
 }
+
+// Token tiles of the two expert GEMMs for a batch of T tokens (an expert sees
+// at most T rows, so a small batch gets small tiles and a deeper ring).
+int tile_gateup_for(int64_t T) { return T <= 64 ? 64 : 128; }
+int tile_down_for(int64_t T) { return T <= 64 ? 64 : (T <= 128 ? 128 : 256); }
 
 // --------------------------------------------------------- CUDA-core path --
 __device__ __forceinline__ int expert_of_row(const int32_t* offsets, int N, int64_t r) {
@@ -535,18 +548,22 @@ cudaError_t launch_simt(const Shape& sh, const void* x_perm, const int32_t* offs
 
 }  // namespace
 
-// out[T, M] (fp32) = b[T, K] (bf16) * a[M, K]^T (bf16) on the tensor cores, run
-// as one "expert" of the grouped kernel's down variant. M is a multiple of 128
-// and K of 64. plan is a device int32[4] holding {0, T, 0, ceil(T / kTileDown)}
-// (that expert's row offsets, then its token-tile prefix).
+// Chunked dense GEMM on the tensor cores, run as one "expert" of the grouped
+// kernel's down variant: for each contraction chunk c of kb_chunk * 64
+// elements, out[t, c * M + i] = sum over k in chunk c of b[t, k] * a[i, k]
+// (fp32, bf16 inputs). M is a multiple of 128 and K of kb_chunk * 64. Every
+// chunk starts a fresh accumulator, which bounds the accumulation chain the
+// tensor cores' fp32 adder runs through. plan is a device int32[4] holding
+// {0, T, 0, ceil(T / kTileDown)} (the expert's rows, then its token tiles).
 cudaError_t launch_dense_gemm_tc(const void* a, int64_t M, const void* b, int64_t T,
-                                 int64_t K, float* out, const int32_t* plan,
-                                 int32_t* err, cudaStream_t st) {
+                                 int64_t K, int kb_chunk, float* out,
+                                 const int32_t* plan, int32_t* err, cudaStream_t st) {
   CUtensorMap am, b16, b128;
   if (!make_map(&am, a, (uint64_t)M, (uint64_t)K, BM) ||
       !make_map(&b16, b, (uint64_t)T, (uint64_t)K, 16) ||
       !make_map(&b128, b, (uint64_t)T, (uint64_t)K, 128))
     return cudaErrorInvalidValue;
+  const int chunks = (int)(K / BK) / kb_chunk;
   GemmArgs g;
   g.offsets = plan;
   g.tile_start = plan + 2;
@@ -554,9 +571,12 @@ cudaError_t launch_dense_gemm_tc(const void* a, int64_t M, const void* b, int64_
   g.err = err;
   g.N = 1;
   g.num_kb = (int)(K / BK);
-  g.out_cols = (int)M;
-  g.m_tiles = (int)(M / BM);
-  return launch_tc<false>(am, am, b16, b128, g, st);
+  g.out_cols = (int)M * chunks;
+  g.m_tiles = (int)(M / BM) * chunks;
+  g.a_rows = (int)M;
+  g.mt_chunk = (int)(M / BM);
+  g.kb_chunk = kb_chunk;
+  return launch_tc<false, kTileDown>(am, am, b16, b128, g, st);
 }
 
 bool expert_ffn_uses_tensor_cores(const Shape& sh) {
@@ -592,8 +612,9 @@ cudaError_t launch_expert_ffn(const Shape& sh, const void* x_perm,
       make_map(&h128, h, rows_cap, (uint64_t)sh.F, 128);
   if (!ok) return cudaErrorInvalidValue;
 
+  const int tgu = tile_gateup_for(sh.T), tdn = tile_down_for(sh.T);
   cudaError_t e = launch_pdl(gemm_plan_kernel, dim3(1), dim3(1024), 0, st, offsets,
-                             (int)sh.N, tile_start);
+                             (int)sh.N, tgu, tdn, tile_start);
   if (e != cudaSuccess) return e;
 
   GemmArgs gu;
@@ -605,7 +626,11 @@ cudaError_t launch_expert_ffn(const Shape& sh, const void* x_perm,
   gu.num_kb = (int)(sh.d / BK);
   gu.out_cols = (int)sh.F;
   gu.m_tiles = (int)(sh.F / BM);
-  e = launch_tc<true>(wg_map, wu_map, x16, x128, gu, st);
+  gu.a_rows = gu.out_cols;
+  gu.mt_chunk = gu.m_tiles;
+  gu.kb_chunk = gu.num_kb;
+  e = tgu == 64 ? launch_tc<true, 64>(wg_map, wu_map, x16, x128, gu, st)
+                : launch_tc<true, 128>(wg_map, wu_map, x16, x128, gu, st);
   if (e != cudaSuccess) return e;
 
   GemmArgs dn = gu;
@@ -614,7 +639,12 @@ cudaError_t launch_expert_ffn(const Shape& sh, const void* x_perm,
   dn.num_kb = (int)(sh.F / BK);
   dn.out_cols = (int)sh.d;
   dn.m_tiles = (int)(sh.d / BM);
-  return launch_tc<false>(wd_map, wd_map, h16, h128, dn, st);
+  dn.a_rows = dn.out_cols;
+  dn.mt_chunk = dn.m_tiles;
+  dn.kb_chunk = dn.num_kb;
+  if (tdn == 64) return launch_tc<false, 64>(wd_map, wd_map, h16, h128, dn, st);
+  if (tdn == 128) return launch_tc<false, 128>(wd_map, wd_map, h16, h128, dn, st);
+  return launch_tc<false, 256>(wd_map, wd_map, h16, h128, dn, st);
 }
 
 }  // namespace moe

@@ -24,7 +24,7 @@ WsLayout ws_layout(const Shape& sh) {
   const size_t Tk = (size_t)(sh.T * sh.k);
   L.header = take(256);
   size_t part = (size_t)router_splits(sh) * sh.T * sh.E;
-  const size_t tc_part = (size_t)sh.T * router_planes_rows(sh);
+  const size_t tc_part = (size_t)sh.T * router_tc_chunks(sh) * router_planes_rows(sh);
   if (router_uses_tensor_cores(sh) && tc_part > part) part = tc_part;
   L.logits = take(part * sizeof(float));
   L.planes = take(router_uses_tensor_cores(sh)
@@ -129,6 +129,11 @@ moe_status_t run_layer(const Shape& sh, const void* x, const float* w_router,
 }
 
 }  // namespace
+
+namespace moe {
+// Configuration checks shared with the entry points defined in other files.
+moe_status_t shape_from_config(const moe_config_t* c, Shape* sh) { return make_shape(c, sh); }
+}  // namespace moe
 
 extern "C" {
 

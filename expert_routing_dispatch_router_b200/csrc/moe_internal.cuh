@@ -77,10 +77,11 @@ cudaError_t launch_combine(const Shape& sh, const void* x, const void* y_perm,
                            const int32_t* idx, const float* gate,
                            const int32_t* slot_row, void* out, cudaStream_t st);
 cudaError_t launch_dense_gemm_tc(const void* a, int64_t M, const void* b, int64_t T,
-                                 int64_t K, float* out, const int32_t* plan,
-                                 int32_t* err, cudaStream_t st);
+                                 int64_t K, int kb_chunk, float* out,
+                                 const int32_t* plan, int32_t* err, cudaStream_t st);
 bool router_uses_tensor_cores(const Shape& sh);
 int64_t router_planes_rows(const Shape& sh);   // 3E rounded up to 128
+int router_tc_chunks(const Shape& sh);         // contraction chunks of that router
 int router_launch_count(const Shape& sh);
 int expert_ffn_launch_count(const Shape& sh);
 int dispatch_launch_count(const Shape& sh);

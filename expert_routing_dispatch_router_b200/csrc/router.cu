@@ -189,8 +189,8 @@ __device__ __forceinline__ uint32_t ord_key(float f) {
 
 template <int PL>
 __global__ void __launch_bounds__(256)
-    topk_kernel(const float* __restrict__ part, int nsplit, int64_t row_stride,
-                int64_t split_stride,
+    topk_kernel(const float* __restrict__ part, int n_outer, int64_t outer_stride,
+                int n_inner, int64_t inner_stride, int64_t row_stride,
                 const float* __restrict__ bias, float* __restrict__ logits_out,
                 int32_t* __restrict__ idx_out, float* __restrict__ gate_out,
                 uint8_t* __restrict__ flags, int64_t T, int E, int k) {
@@ -200,18 +200,21 @@ __global__ void __launch_bounds__(256)
   griddep_launch_dependents();
   if (t >= T) return;
 
-  // logits = partial sums added in split order (fixed, so reproducible); the
-  // loads of several splits are issued together
+  // logits = partial sums added in a fixed order (outer, then inner index),
+  // so results are reproducible; the loads of several partials are issued
+  // together
   float lg[PL], key[PL];
 #pragma unroll
   for (int i = 0; i < PL; ++i) lg[i] = 0.f;
   const float* pt = part + t * row_stride + lane;
-  const int64_t zstride = split_stride;
+  for (int zo = 0; zo < n_outer; ++zo) {
 #pragma unroll 4
-  for (int z = 0; z < nsplit; ++z) {
+    for (int zi = 0; zi < n_inner; ++zi) {
+      const float* pz = pt + zo * outer_stride + zi * inner_stride;
 #pragma unroll
-    for (int i = 0; i < PL; ++i)
-      if (lane + 32 * i < E) lg[i] += pt[z * zstride + 32 * i];
+      for (int i = 0; i < PL; ++i)
+        if (lane + 32 * i < E) lg[i] += pz[32 * i];
+    }
   }
 #pragma unroll
   for (int i = 0; i < PL; ++i) {
@@ -286,14 +289,14 @@ __global__ void __launch_bounds__(256)
 }
 
 template <int PL>
-void launch_topk(const float* part, int nsplit, int64_t row_stride,
-                 int64_t split_stride, const float* bias,
+void launch_topk(const float* part, int n_outer, int64_t outer_stride, int n_inner,
+                 int64_t inner_stride, int64_t row_stride, const float* bias,
                  float* logits, int32_t* idx, float* gate, uint8_t* flags,
                  int64_t T, int E, int k, cudaStream_t st) {
   const int warps = 8;
   const unsigned grid = (unsigned)((T + warps - 1) / warps);
-  launch_pdl(topk_kernel<PL>, dim3(grid), dim3(warps * 32), 0, st, part, nsplit,
-             row_stride, split_stride, bias,
+  launch_pdl(topk_kernel<PL>, dim3(grid), dim3(warps * 32), 0, st, part, n_outer,
+             outer_stride, n_inner, inner_stride, row_stride, bias,
              logits, idx, gate, flags, T, E, k);
 }
 
@@ -355,6 +358,17 @@ constexpr int64_t kTcRouterMinTokens = 512;
 
 int64_t router_planes_rows(const Shape& sh) { return (3 * sh.E + 127) / 128 * 128; }
 
+// The tensor-core router restarts its fp32 accumulation every 1024 contraction
+// elements (16 blocks of 64), a chain of 64 MMA steps per partial.
+static int router_kb_chunk(const Shape& sh) {
+  const int kb = (int)(sh.d / 64);
+  int c = kb < 16 ? kb : 16;
+  while (kb % c != 0) --c;
+  return c;
+}
+
+int router_tc_chunks(const Shape& sh) { return (int)(sh.d / 64) / router_kb_chunk(sh); }
+
 bool router_uses_tensor_cores(const Shape& sh) {
   return sh.bf16 && sh.d % 128 == 0 && sh.T >= kTcRouterMinTokens &&
          router_planes_rows(sh) <= 4096;
@@ -378,8 +392,8 @@ cudaError_t launch_router(const Shape& sh, const void* x, const float* w_r,
                           float* gate, uint8_t* flags, float* logits_out,
                           void* planes, int32_t* plan, int32_t* err,
                           cudaStream_t st) {
-  int nsplit;
-  int64_t row_stride, split_stride;
+  int n_outer, n_inner;
+  int64_t outer_stride, inner_stride, row_stride;
   cudaError_t e;
   if (router_uses_tensor_cores(sh)) {
     const int64_t Ep = router_planes_rows(sh);
@@ -390,13 +404,17 @@ cudaError_t launch_router(const Shape& sh, const void* x, const float* w_r,
                    reinterpret_cast<const float4*>(w_r), sh.E, sh.d, Ep,
                    static_cast<uint2*>(planes), plan, sh.T, kTileDown);
     if (e != cudaSuccess) return e;
-    e = launch_dense_gemm_tc(planes, Ep, x, sh.T, sh.d, part, plan, err, st);
+    e = launch_dense_gemm_tc(planes, Ep, x, sh.T, sh.d, router_kb_chunk(sh), part, plan,
+                             err, st);
     if (e != cudaSuccess) return e;
-    nsplit = 3;
-    row_stride = Ep;
-    split_stride = sh.E;
+    // part[t, c * Ep + p * E + e]: chunk c, plane p (hi, mid, lo)
+    n_outer = router_tc_chunks(sh);
+    outer_stride = Ep;
+    n_inner = 3;
+    inner_stride = sh.E;
+    row_stride = (int64_t)n_outer * Ep;
   } else {
-    nsplit = router_splits(sh);
+    const int nsplit = router_splits(sh);
     int64_t kps = (sh.d + nsplit - 1) / nsplit;
     kps = (kps + RK - 1) / RK * RK;
     dim3 grid((unsigned)((sh.E + RE - 1) / RE), (unsigned)((sh.T + RT - 1) / RT),
@@ -409,14 +427,17 @@ cudaError_t launch_router(const Shape& sh, const void* x, const float* w_r,
       e = launch_pdl(router_logits_kernel<float>, grid, dim3(kRouterThreads), 0, st,
                      static_cast<const float*>(x), w_r, part, sh.T, sh.d, sh.E, kps);
     if (e != cudaSuccess) return e;
+    n_outer = nsplit;
+    outer_stride = sh.T * sh.E;
+    n_inner = 1;
+    inner_stride = 0;
     row_stride = sh.E;
-    split_stride = sh.T * sh.E;
   }
   const int pl = (int)((sh.E + 31) / 32);
   const int E = (int)sh.E, k = (int)sh.k;
-#define MOE_TOPK(P)                                                                    \
-  launch_topk<P>(part, nsplit, row_stride, split_stride, bias, logits_out, idx, gate, \
-                 flags, sh.T, E, k, st)
+#define MOE_TOPK(P)                                                                 \
+  launch_topk<P>(part, n_outer, outer_stride, n_inner, inner_stride, row_stride, bias, \
+                 logits_out, idx, gate, flags, sh.T, E, k, st)
   if (pl <= 1)
     MOE_TOPK(1);
   else if (pl <= 2)
@@ -430,6 +451,47 @@ cudaError_t launch_router(const Shape& sh, const void* x, const float* w_r,
   else
     MOE_TOPK(32);
 #undef MOE_TOPK
+  return cudaGetLastError();
+}
+
+// The CUDA-core router with a caller-chosen number of contraction splits and
+// caller-provided scratch `part` of nsplit * T * E floats (used by the
+// entry point that allocates nothing).
+cudaError_t launch_router_simt(const Shape& sh, const void* x, const float* w_r,
+                               const float* bias, float* part, int nsplit,
+                               int32_t* idx, float* gate, uint8_t* flags,
+                               float* logits_out, cudaStream_t st) {
+  int64_t kps = (sh.d + nsplit - 1) / nsplit;
+  kps = (kps + RK - 1) / RK * RK;
+  dim3 grid((unsigned)((sh.E + RE - 1) / RE), (unsigned)((sh.T + RT - 1) / RT),
+            (unsigned)nsplit);
+  cudaError_t e;
+  if (sh.bf16)
+    e = launch_pdl(router_logits_kernel<__nv_bfloat16>, grid, dim3(kRouterThreads), 0, st,
+                   static_cast<const __nv_bfloat16*>(x), w_r, part, sh.T, sh.d, sh.E, kps);
+  else
+    e = launch_pdl(router_logits_kernel<float>, grid, dim3(kRouterThreads), 0, st,
+                   static_cast<const float*>(x), w_r, part, sh.T, sh.d, sh.E, kps);
+  if (e != cudaSuccess) return e;
+  const int64_t split_stride = sh.T * sh.E;
+  const int pl = (int)((sh.E + 31) / 32);
+  const int E = (int)sh.E, k = (int)sh.k;
+#define MOE_TOPK_S(P)                                                                 \
+  launch_topk<P>(part, nsplit, split_stride, 1, 0, sh.E, bias, logits_out, idx, gate, \
+                 flags, sh.T, E, k, st)
+  if (pl <= 1)
+    MOE_TOPK_S(1);
+  else if (pl <= 2)
+    MOE_TOPK_S(2);
+  else if (pl <= 4)
+    MOE_TOPK_S(4);
+  else if (pl <= 8)
+    MOE_TOPK_S(8);
+  else if (pl <= 16)
+    MOE_TOPK_S(16);
+  else
+    MOE_TOPK_S(32);
+#undef MOE_TOPK_S
   return cudaGetLastError();
 }
 
