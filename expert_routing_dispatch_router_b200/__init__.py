@@ -96,6 +96,7 @@ def lib():
             "moe_layer_forward": ([C, P, P, P, P, P, P, P, P, P, sz, P], i32),
             "moe_layer_forward_host": ([C, P, P, P, P, P, P, P, P, P, sz, P], i32),
             "moe_read_device_error": ([P, P, P], i32),
+            "moe_route_noalloc": ([C, P, P, P, P, P, P, P, P], i32),
             "moe_layer_launch_count": ([C], ctypes.c_int32),
             "moe_status_string": ([i32], ctypes.c_char_p),
         }
@@ -165,6 +166,29 @@ def route(shape: LayerShape, x, w_router, bias, ws, logits=None, flags=None,
                          ws.numel(), _stream(stream))
     _check("moe_route", st)
     return idx, gate
+
+
+def route_noalloc(shape: LayerShape, x, w_router, bias, topk_idx, topk_gate,
+                  logits=None, flags=None, stream=None):
+    """moe_route without a workspace, for callers that cannot allocate device
+    memory: every output is caller-provided and the library's own fixed
+    scratch array is used (T * E <= 4194304). Calls sharing a device must not
+    overlap on the GPU."""
+    T, E, k = shape.T, shape.E, shape.top_k
+    _need(x, "x", shape.act_dtype, (T, shape.d))
+    _need(w_router, "w_router", torch.float32, (E, shape.d))
+    _need(bias, "bias", torch.float32, (E,))
+    _need(topk_idx, "topk_idx", torch.int32, (T, k))
+    _need(topk_gate, "topk_gate", torch.float32, (T, k))
+    if logits is not None:
+        _need(logits, "logits", torch.float32, (T, E))
+    if flags is not None:
+        _need(flags, "flags", torch.uint8, (T,))
+    st = lib().moe_route_noalloc(ctypes.byref(shape.c()), _ptr(x), _ptr(w_router),
+                                 _ptr(bias), _ptr(logits), _ptr(topk_idx),
+                                 _ptr(topk_gate), _ptr(flags), _stream(stream))
+    _check("moe_route_noalloc", st)
+    return topk_idx, topk_gate
 
 
 def dispatch(shape: LayerShape, x, topk_idx, ws, stream=None):

@@ -166,6 +166,27 @@ moe_status_t moe_layer_forward_host(const moe_config_t* cfg, const void* x_host,
                                     int32_t* counts_host, void* ws,
                                     size_t ws_bytes, moe_stream_t stream);
 
+/* moe_route without a workspace, for callers that cannot allocate device
+ * memory: code running inside an allocator or memory pool that owns the whole
+ * device, plugins whose host forbids allocation after start-up, and paths
+ * that must never wait on an allocator. The pages have no counterpart of this
+ * call; it exists for those callers only.
+ *  Same arguments, layouts and results as moe_route, minus ws/ws_bytes (it
+ *  always runs the CUDA-core router). It allocates nothing: its scratch is
+ *  one 16 MiB array inside the library, held by every GPU that loads the
+ *  library until the process exits.
+ *  Limit: T * (n_routed + n_zero) <= 4194304; larger problems return
+ *  MOE_ERR_UNSUPPORTED before anything is launched.
+ *  The first call on a device (with that device current) looks up the
+ *  array's address once; make it before any stream capture on that device.
+ *  All calls on a device share the array: calls that overlap on the GPU
+ *  (other streams or host threads) race and must be ordered by the caller. */
+moe_status_t moe_route_noalloc(const moe_config_t* cfg, const void* x,
+                               const float* w_router, const float* bias,
+                               float* logits, int32_t* topk_idx,
+                               float* topk_gate, uint8_t* flags,
+                               moe_stream_t stream);
+
 /* Waits for `stream`, then reads and clears the device-side error word in ws.
  * *code_out (may be NULL) gets 0 when no check failed, else a nonzero code
  * (1 = a bounded wait in the expert GEMM ran out, 2 = a routing slot held an
