@@ -16,6 +16,7 @@ and the only collectives are the timing barrier and the max over ranks.
 of the same workload on this machine's host cores; rank 0 only.
 """
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -44,6 +45,34 @@ def peaks():
                 "source": "measured"}
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
             "source": "fallback"}
+
+
+KERNEL_SOURCES = ("expert_ffn.cu", "sm100_ptx.cuh", "moe_internal.cuh")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "grouped_gemm_tc_traffic.json")
+
+
+def kernel_source_digest():
+    """Digest of the expert-GEMM sources; a recorded ncu traffic figure is only
+    reported while the kernel it was taken on is unchanged."""
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "expert_routing_dispatch_router_b200", "csrc",
+                               name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(config_name, units):
+    """ncu dram bytes (read + write) of one gate/up + down launch pair, scaled
+    from the recorded capture by the touched experts, or None."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    with open(TRAFFIC_FILE) as f:
+        rec = json.load(f)
+    entry = rec.get(config_name)
+    if not entry or entry.get("source_digest") != kernel_source_digest():
+        return None
+    return entry["dram_bytes_per_touched_expert"] * units
 
 
 def workload_name(sh):
@@ -339,8 +368,7 @@ def run_gpu(args, sh):
                 "kernel": "moe_expert_ffn: grouped_gemm_tc gate/up + down (+ plan)",
                 "algorithmic_bytes": b_ffn,
                 "peak_source": pk["source"] + " hbm_gbs (burst copy)"}
-        if args.traffic_bytes:
-            roof["traffic"] = args.traffic_bytes
+        roof["traffic"] = measured_traffic(sh.name, U)
 
     if rank == 0:
         line = {
@@ -378,8 +406,6 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-tokens", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--traffic-bytes", type=float, default=None,
-                    help="ncu dram bytes per launch of the dominant kernel pair")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -96,20 +96,25 @@ constexpr int BK = 64;   // contraction elements per stage: 128-byte rows
 constexpr int kThreads = 192;
 constexpr uint32_t kTileBytes = BM * BK * 2;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kAccStride = 256;  // TMEM columns per accumulator buffer
+constexpr uint32_t kAccStride = 256;  // TMEM columns per accumulator buffer (2 buffers)
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
-// Gate/up: two weight tiles (W_gate, W_up rows) x up to 128 tokens, two fp32
-// accumulators of <= 128 columns. Down: one weight tile x up to 256 tokens,
-// one accumulator of <= 256 columns. Either way a TMEM buffer is 256 columns
-// and there are two of them. Token tiles are sized to the batch on the host
-// (an expert sees at most T rows): small tiles leave room for more stages, so
-// a decode step keeps more weight bytes in flight.
+// Gate/up: two weight tiles (W_gate, W_up rows) x up to BN tokens, two fp32
+// accumulators of BN columns. Down: one weight tile x up to BN tokens, one
+// accumulator of BN columns. When one accumulator set fits in 256 TMEM
+// columns there are two sets, so the epilogue of a tile overlaps the MMAs of
+// the next; the 256-token gate/up tile fills all 512 columns with one set and
+// the MMAs wait for its epilogue (short against its 64-block main loop).
+// Token tiles are sized to the batch on the host (an expert sees at most T
+// rows): small tiles leave room for more stages, so a decode step keeps more
+// weight bytes in flight, and large tiles halve the bytes each FLOP needs.
 template <bool GATEUP, int BN_>
 struct Cfg {
   static constexpr int kNumA = GATEUP ? 2 : 1;
   static constexpr int BN = BN_;  // max MMA N
-  static_assert(BN % 16 == 0 && BN <= (GATEUP ? 128 : 256), "token tile");
+  static_assert(BN % 16 == 0 && BN <= 256, "token tile");
+  static constexpr uint32_t kAccCols = kNumA * BN;  // columns of one accumulator set
+  static constexpr int kAccBufs = kAccCols <= kAccStride ? 2 : 1;
   static constexpr uint32_t kBBytes = BN * BK * 2;
   static constexpr uint32_t kStageBytes = kNumA * kTileBytes + kBBytes;
   static constexpr int kStages =
@@ -322,7 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ptx::tc_fence_after();
         const uint32_t idesc = ptx::idesc_bf16_f32(BM, un.n_mma);
-        const uint32_t d0 = tmem_base + (uint32_t)acc * kAccStride;
+        const uint32_t d0 = tmem_base + (uint32_t)acc * kAccStride;  // acc = 0 if one set
         for (int kb = 0; kb < args.kb_chunk; ++kb) {
           if (!wait_bounded(full_bar(stage), phase, abort_flag, args.err)) {
             ok = false;
@@ -337,7 +342,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
             ptx::mma_bf16(d0, ptx::desc_k_sw128(a0 + kk * 32), bdesc, idesc, accum);
             if (GATEUP)
-              ptx::mma_bf16(d0 + 128, ptx::desc_k_sw128(a0 + kTileBytes + kk * 32),
+              ptx::mma_bf16(d0 + BN, ptx::desc_k_sw128(a0 + kTileBytes + kk * 32),
                             bdesc, idesc, accum);
           }
           issued = true;
@@ -349,8 +354,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!ok) break;
         ptx::mma_commit(tfull_bar(acc));
-        acc ^= 1;
-        if (acc == 0) acc_phase ^= 1u;
+        if (++acc == C::kAccBufs) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
       }
       if (!ok && issued) {  // the MMAs already issued must finish before TMEM is freed
         ptx::mma_commit(mma_done_bar);
@@ -375,7 +382,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c0 = 0; c0 < un.n_mma; c0 += 16) {
         float g[16], v[16];
         if (GATEUP) {
-          ptx::tmem_ld16x2(tb + c0, tb + 128 + c0, g, v);
+          ptx::tmem_ld16x2(tb + c0, tb + BN + c0, g, v);
           __nv_bfloat16* outp = static_cast<__nv_bfloat16*>(args.out) + obase;
 #pragma unroll
           for (int c = 0; c < 16; ++c)
@@ -393,8 +400,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(tempty_bar(acc));
-      acc ^= 1;
-      if (acc == 0) acc_phase ^= 1u;
+      if (++acc == C::kAccBufs) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
     }
   }
 
@@ -454,7 +463,7 @@ cudaError_t launch_tc(const CUtensorMap& a0, const CUtensorMap& a1,
 
 // Token tiles of the two expert GEMMs for a batch of T tokens (an expert sees
 // at most T rows, so a small batch gets small tiles and a deeper ring).
-int tile_gateup_for(int64_t T) { return T <= 64 ? 64 : 128; }
+int tile_gateup_for(int64_t T) { return T <= 64 ? 64 : (T <= 1024 ? 128 : 256); }
 int tile_down_for(int64_t T) { return T <= 64 ? 64 : (T <= 128 ? 128 : 256); }
 
 // --------------------------------------------------------- CUDA-core path --
@@ -629,8 +638,9 @@ cudaError_t launch_expert_ffn(const Shape& sh, const void* x_perm,
   gu.a_rows = gu.out_cols;
   gu.mt_chunk = gu.m_tiles;
   gu.kb_chunk = gu.num_kb;
-  e = tgu == 64 ? launch_tc<true, 64>(wg_map, wu_map, x16, x128, gu, st)
-                : launch_tc<true, 128>(wg_map, wu_map, x16, x128, gu, st);
+  e = tgu == 64    ? launch_tc<true, 64>(wg_map, wu_map, x16, x128, gu, st)
+      : tgu == 128 ? launch_tc<true, 128>(wg_map, wu_map, x16, x128, gu, st)
+                   : launch_tc<true, 256>(wg_map, wu_map, x16, x128, gu, st);
   if (e != cudaSuccess) return e;
 
   GemmArgs dn = gu;

@@ -85,6 +85,9 @@ CONFIGS: Dict[str, MoEShape] = {
                                n_zero=8, top_k=8, ffn=1024),
     "profile_prefill": MoEShape("profile_prefill", T=4096, d=4096, n_routed=32,
                                 n_zero=8, top_k=8, ffn=1024, routing="zipf"),
+    # the large-expert layer's density (~270 rows per expert), 32 experts
+    "profile_large_e": MoEShape("profile_large_e", T=1024, d=6144, n_routed=32,
+                                n_zero=8, top_k=12, ffn=2048),
 }
 
 SWEEP_T = (1, 8, 64, 512, 4096, 32768)
