@@ -42,6 +42,12 @@ class MoEConfig(ctypes.Structure):
                 ("act_dtype", ctypes.c_int32), ("routed_scale", ctypes.c_float)]
 
 
+class MoEPIDParams(ctypes.Structure):
+    _fields_ = [("target_routed_share", ctypes.c_float), ("kp", ctypes.c_float),
+                ("ki", ctypes.c_float), ("kd", ctypes.c_float),
+                ("max_step", ctypes.c_float)]
+
+
 @dataclass(frozen=True)
 class LayerShape:
     """Sizes of one layer call (mirrors moe_config_t)."""
@@ -97,6 +103,7 @@ def lib():
             "moe_layer_forward_host": ([C, P, P, P, P, P, P, P, P, P, sz, P], i32),
             "moe_read_device_error": ([P, P, P], i32),
             "moe_route_noalloc": ([C, P, P, P, P, P, P, P, P], i32),
+            "moe_bias_pid_update": ([C, P, P, P, ctypes.POINTER(MoEPIDParams), P], i32),
             "moe_layer_launch_count": ([C], ctypes.c_int32),
             "moe_status_string": ([i32], ctypes.c_char_p),
         }
@@ -296,3 +303,18 @@ def read_device_error(ws, stream=None) -> int:
     code = ctypes.c_int32(0)
     lib().moe_read_device_error(_ptr(ws), ctypes.byref(code), _stream(stream))
     return int(code.value)
+
+
+def bias_pid_update(shape: LayerShape, counts, bias, state, target: float, kp: float,
+                    ki: float = 0.0, kd: float = 0.0, max_step: float = 1.0,
+                    stream=None):
+    """One PID step on the zero experts' router bias (in place on `bias` and
+    `state`), from the per-expert counts of the last layer call."""
+    _need(counts, "counts", torch.int32, (shape.E,))
+    _need(bias, "bias", torch.float32, (shape.E,))
+    _need(state, "state", torch.float64, (2,))
+    prm = MoEPIDParams(target, kp, ki, kd, max_step)
+    st = lib().moe_bias_pid_update(ctypes.byref(shape.c()), _ptr(counts), _ptr(bias),
+                                   _ptr(state), ctypes.byref(prm), _stream(stream))
+    _check("moe_bias_pid_update", st)
+    return bias, state

@@ -8,7 +8,9 @@
 // GEMM (gate/up, then down), warp-specialised for sm_100a:
 //   warp 0      TMA producer: weight tiles and token tiles -> smem ring
 //   warp 1      MMA issuer: tcgen05.mma into TMEM (fp32), tcgen05.commit
-//   warps 2..5  epilogue: tcgen05.ld from TMEM, SwiGLU, bf16 stores
+//   warps 2..9  epilogue: tcgen05.ld from TMEM, SwiGLU, bf16 stores (two
+//               warps per TMEM lane quarter, each taking every other
+//               32-column chunk)
 // The operands are swapped relative to the usual token-major GEMM: 128 rows
 // of an expert's weight matrix fill the MMA's M = 128 and the expert's tokens
 // (up to 128 per tile, rounded up to a multiple of 16) are its N. A decode
@@ -93,7 +95,10 @@ __global__ void __launch_bounds__(1024)
 // ------------------------------------------------------- tensor-core path --
 constexpr int BM = 128;  // weight rows per tile (MMA M)
 constexpr int BK = 64;   // contraction elements per stage: 128-byte rows
-constexpr int kThreads = 192;
+// warp 0: TMA producer, warp 1: MMA issuer, warps 2..9: epilogue (two warps
+// per TMEM lane quarter, splitting the accumulator columns)
+constexpr int kThreads = 320;
+constexpr int kEpiWarps = 8;
 constexpr uint32_t kTileBytes = BM * BK * 2;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccStride = 256;  // TMEM columns per accumulator buffer (2 buffers)
@@ -232,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       ptx::mbar_init(tfull_bar(b), 1);
-      ptx::mbar_init(tempty_bar(b), 4);
+      ptx::mbar_init(tempty_bar(b), kEpiWarps);
     }
     ptx::mbar_init(mma_done_bar, 1);
     *abort_flag = 0;
@@ -366,7 +371,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // -------------------------------------------------------- epilogue --
-    const int ew = warp & 3;  // TMEM lane quarter this warp may access
+    const int ew = warp & 3;          // TMEM lane quarter this warp may access
+    const int eh = (warp - 2) >> 2;   // which half of the column chunks
     const int lrow = ew * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -379,21 +385,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                           (uint32_t)acc * kAccStride;
       const int64_t col = (int64_t)un.m * BM + lrow;
       const int64_t obase = (int64_t)un.row0 * args.out_cols + col;
-      for (int c0 = 0; c0 < un.n_mma; c0 += 16) {
-        float g[16], v[16];
+      // 32-column chunks, alternating between the two warps of this quarter
+      for (int c0 = 32 * eh; c0 < un.n_mma; c0 += 64) {
+        float g[32], v[32];
         if (GATEUP) {
-          ptx::tmem_ld16x2(tb + c0, tb + BN + c0, g, v);
+          ptx::tmem_ld32x2(tb + c0, tb + BN + c0, g, v);
           __nv_bfloat16* outp = static_cast<__nv_bfloat16*>(args.out) + obase;
 #pragma unroll
-          for (int c = 0; c < 16; ++c)
+          for (int c = 0; c < 32; ++c)
             if (c0 + c < un.n_valid)
               outp[(int64_t)(c0 + c) * args.out_cols] =
                   __float2bfloat16_rn(silu_f(g[c]) * v[c]);
         } else {
-          ptx::tmem_ld16(tb + c0, g);
+          ptx::tmem_ld32(tb + c0, g);
           float* outp = static_cast<float*>(args.out) + obase;
 #pragma unroll
-          for (int c = 0; c < 16; ++c)
+          for (int c = 0; c < 32; ++c)
             if (c0 + c < un.n_valid) outp[(int64_t)(c0 + c) * args.out_cols] = g[c];
         }
       }
@@ -412,6 +419,273 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// -------------------------------------------- CTA-pair path (cta_group::2) --
+// For batches with many rows per expert the same GEMMs run on pairs of CTAs
+// (a 2-CTA cluster on one GPC). A unit is (expert, 256 weight rows, up to 256
+// tokens): each CTA loads 128 of the weight rows and half of the token rows,
+// the leader issues M = 256 MMAs that read both CTAs' shared memory, and each
+// CTA's TMEM receives the accumulators of its own 128 weight rows for all the
+// unit's tokens. Per FLOP this loads half the shared-memory bytes of the
+// single-CTA kernel, and the two CTAs that share every tile sit on one die.
+//
+// Protocol (barriers at the same offsets in both CTAs):
+//   full[s]   leader's: armed by the leader's producer with both CTAs' bytes;
+//             both CTAs' TMA loads complete on it (cta_group::2 loads)
+//   empty[s]  both: the leader's MMA commit arrives on both (multicast commit)
+//   tfull[b]  both: the leader's commit after a unit's last MMA
+//   tempty[b] leader's, 16 arrivals: 8 epilogue warps here + 8 in the peer
+template <bool GATEUP>
+struct PairCfg {
+  static constexpr int kNumA = GATEUP ? 2 : 1;
+  static constexpr int BN = 256;   // token columns of a unit (both CTAs)
+  static constexpr int BNH = 128;  // token rows one CTA loads, at most
+  static constexpr uint32_t kStageBytes = kNumA * kTileBytes + BNH * BK * 2;
+  static constexpr int kStages = (int)(204800 / kStageBytes);  // 4 or 6
+  static constexpr uint32_t kAccCols = kNumA * BN;             // 512 or 256
+  static constexpr int kAccBufs = kAccCols <= kAccStride ? 2 : 1;
+  static constexpr uint32_t kBarOff = kStages * kStageBytes;
+  static constexpr uint32_t kTabOff = kBarOff + 256;
+  static constexpr uint32_t kSmemBytes = 1024 + kTabOff + 2 * 4 * (kMaxExperts + 1);
+};
+
+// Busy wait of about `ns` nanoseconds (lets in-flight copies land on abort).
+__device__ __forceinline__ void settle_ns(uint64_t ns) {
+  const uint64_t t0 = ptx::global_timer_ns();
+  while (ptx::global_timer_ns() - t0 < ns) {
+  }
+}
+
+template <bool GATEUP>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0,
+                             const __grid_constant__ CUtensorMap tmA1,
+                             const __grid_constant__ CUtensorMap tmB16,
+                             const __grid_constant__ CUtensorMap tmB128,
+                             const GemmArgs args) {
+  using C = PairCfg<GATEUP>;
+  constexpr int S = C::kStages;
+  constexpr int BN = C::BN;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = ptx::smem_addr(smem);
+  const uint32_t bars = sbase + C::kBarOff;
+  auto full_bar = [&](int s) { return bars + 8u * s; };
+  auto empty_bar = [&](int s) { return bars + 8u * (S + s); };
+  auto tfull_bar = [&](int b) { return bars + 8u * (2 * S + b); };
+  auto tempty_bar = [&](int b) { return bars + 8u * (2 * S + 2 + b); };
+  const uint32_t mma_done_bar = bars + 8u * (2 * S + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + 8 * (2 * S + 5));
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* s_tiles = reinterpret_cast<int*>(smem + C::kTabOff);
+  int* s_offs = s_tiles + (kMaxExperts + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int N = args.N;
+  const uint32_t rank = ptx::cluster_ctarank();
+  const bool leader = rank == 0;
+  const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      ptx::mbar_init(full_bar(s), 1);
+      ptx::mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(tfull_bar(b), 1);
+      ptx::mbar_init(tempty_bar(b), 2 * kEpiWarps);
+    }
+    ptx::mbar_init(mma_done_bar, 1);
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    ptx::prefetch_tensormap(&tmA0);
+    if (GATEUP) ptx::prefetch_tensormap(&tmA1);
+    ptx::prefetch_tensormap(&tmB16);
+    ptx::prefetch_tensormap(&tmB128);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc_pair(ptx::smem_addr(tmem_slot), kTmemCols);
+    ptx::tmem_relinquish_pair();
+  }
+  griddep_wait();
+  griddep_launch_dependents();
+  for (int i = threadIdx.x; i <= N; i += blockDim.x) {
+    s_tiles[i] = args.tile_start[i];
+    s_offs[i] = args.offsets[i];
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::cluster_sync();  // both CTAs' barriers exist before any remote arrive
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
+  const int total_units = s_tiles[N] * args.m_tiles;
+
+  if (warp == 0) {
+    // ---------------------------------------------------- TMA producer --
+    if (lane == 0) {
+      const uint64_t pol_first = ptx::policy_evict_first();
+      const uint64_t pol_last = ptx::policy_evict_last();
+      const uint64_t pol_normal = ptx::policy_evict_normal();
+      int stage = 0;
+      uint32_t phase = 0, armed = 0, armed_par = 0;
+      bool ok = true, issued = false;
+      for (int u = cid; u < total_units && ok; u += ncl) {
+        const Unit un = decode_unit<BN>(u, s_tiles, s_offs, N, args.m_tiles);
+        const int n_pair = (un.n_valid + 31) & ~31;  // MMA N; each CTA holds half
+        const int half = n_pair >> 1;
+        const int arow = un.e * args.a_rows + un.m * 2 * BM + (int)rank * BM;
+        const int brow = un.row0 + (int)rank * half;
+        const uint32_t bytes = 2u * (C::kNumA * kTileBytes + (uint32_t)half * 128u);
+        const uint64_t pol_w = un.ntiles == 1 ? pol_first : pol_normal;
+        const uint64_t pol_x = un.ntiles == 1 ? pol_last : pol_normal;
+        for (int kb = 0; kb < args.num_kb; ++kb) {
+          if (!wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, args.err)) {
+            ok = false;
+            break;
+          }
+          if (leader) ptx::mbar_arrive_expect_tx(full_bar(stage), bytes);
+          const uint32_t lbar = ptx::map_to_rank(full_bar(stage), 0);
+          const uint32_t a0 = sbase + stage * C::kStageBytes;
+          ptx::tma_load_2d_pair(&tmA0, a0, lbar, kb * BK, arow, pol_w);
+          if (GATEUP) ptx::tma_load_2d_pair(&tmA1, a0 + kTileBytes, lbar, kb * BK, arow, pol_w);
+          const uint32_t b0 = a0 + C::kNumA * kTileBytes;
+          int j = 0;
+          for (; j + 128 <= half; j += 128)
+            ptx::tma_load_2d_pair(&tmB128, b0 + j * 128u, lbar, kb * BK, brow + j, pol_x);
+          for (; j < half; j += 16)
+            ptx::tma_load_2d_pair(&tmB16, b0 + j * 128u, lbar, kb * BK, brow + j, pol_x);
+          issued = true;
+          armed |= 1u << stage;
+          armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        // let our own loads land before the CTA goes away: the leader can see
+        // them on its full barriers, the peer's complete on the leader's
+        if (leader) {
+          for (int s = 0; s < S; ++s)
+            if ((armed >> s) & 1u) wait_cleanup(full_bar(s), (armed_par >> s) & 1u);
+        } else if (issued) {
+          settle_ns(2000000);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // --------------------------------------------- MMA issuer (leader) --
+    if (lane == 0 && leader) {
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true, issued = false;
+      for (int u = cid; u < total_units && ok; u += ncl) {
+        const Unit un = decode_unit<BN>(u, s_tiles, s_offs, N, args.m_tiles);
+        const int n_pair = (un.n_valid + 31) & ~31;
+        if (!wait_bounded(tempty_bar(acc), acc_phase ^ 1u, abort_flag, args.err)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t idesc = ptx::idesc_bf16_f32(2 * BM, n_pair);
+        const uint32_t d0 = tmem_base + (uint32_t)acc * kAccStride;
+        for (int kb = 0; kb < args.num_kb; ++kb) {
+          if (!wait_bounded(full_bar(stage), phase, abort_flag, args.err)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t a0 = sbase + stage * C::kStageBytes;
+          const uint32_t b0 = a0 + C::kNumA * kTileBytes;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t bdesc = ptx::desc_k_sw128(b0 + kk * 32);
+            const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
+            ptx::mma_bf16_pair(d0, ptx::desc_k_sw128(a0 + kk * 32), bdesc, idesc, accum);
+            if (GATEUP)
+              ptx::mma_bf16_pair(d0 + BN, ptx::desc_k_sw128(a0 + kTileBytes + kk * 32),
+                                 bdesc, idesc, accum);
+          }
+          issued = true;
+          ptx::mma_commit_pair(empty_bar(stage));
+          if (++stage == S) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        ptx::mma_commit_pair(tfull_bar(acc));
+        if (++acc == C::kAccBufs) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      if (!ok && issued) {  // MMAs already issued must finish before TMEM is freed
+        ptx::mma_commit_pair(mma_done_bar);
+        wait_cleanup(mma_done_bar, 0);
+      }
+    }
+  } else {
+    // -------------------------------------------------------- epilogue --
+    const int ew = warp & 3;          // TMEM lane quarter
+    const int eh = (warp - 2) >> 2;   // which half of the column chunks
+    const int lrow = ew * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int u = cid; u < total_units; u += ncl) {
+      const Unit un = decode_unit<BN>(u, s_tiles, s_offs, N, args.m_tiles);
+      const int n_pair = (un.n_valid + 31) & ~31;
+      const bool ok = wait_bounded(tfull_bar(acc), acc_phase, abort_flag, args.err);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      ptx::tc_fence_after();
+      const uint32_t tb = tmem_base + (static_cast<uint32_t>(ew * 32) << 16) +
+                          (uint32_t)acc * kAccStride;
+      const int64_t col = (int64_t)un.m * 2 * BM + (int64_t)rank * BM + lrow;
+      const int64_t obase = (int64_t)un.row0 * args.out_cols + col;
+      for (int c0 = 32 * eh; c0 < n_pair; c0 += 64) {
+        float g[32], v[32];
+        if (GATEUP) {
+          ptx::tmem_ld32x2(tb + c0, tb + BN + c0, g, v);
+          __nv_bfloat16* outp = static_cast<__nv_bfloat16*>(args.out) + obase;
+#pragma unroll
+          for (int c = 0; c < 32; ++c)
+            if (c0 + c < un.n_valid)
+              outp[(int64_t)(c0 + c) * args.out_cols] =
+                  __float2bfloat16_rn(silu_f(g[c]) * v[c]);
+        } else {
+          ptx::tmem_ld32(tb + c0, g);
+          float* outp = static_cast<float*>(args.out) + obase;
+#pragma unroll
+          for (int c = 0; c < 32; ++c)
+            if (c0 + c < un.n_valid) outp[(int64_t)(c0 + c) * args.out_cols] = g[c];
+        }
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (leader)
+          ptx::mbar_arrive(tempty_bar(acc));
+        else
+          ptx::mbar_arrive_remote(ptx::map_to_rank(tempty_bar(acc), 0));
+      }
+      if (++acc == C::kAccBufs) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::cluster_sync();  // neither CTA frees TMEM or exits while the pair works
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc_pair(tmem_base, kTmemCols);
   }
 }
 
@@ -461,9 +735,64 @@ cudaError_t launch_tc(const CUtensorMap& a0, const CUtensorMap& a1,
                     C::kSmemBytes, st, a0, a1, b16, b128, args);
 }
 
+// CTA-pair launch: clusters of 2 with programmatic dependent launch, as many
+// pairs as can be resident at once (so the persistent schedule has no tail).
+template <bool GATEUP>
+cudaError_t launch_pair(const CUtensorMap& a0, const CUtensorMap& a1,
+                        const CUtensorMap& b16, const CUtensorMap& b128,
+                        const GemmArgs& args, cudaStream_t st) {
+  using C = PairCfg<GATEUP>;
+  static int grid = 0;
+  if (grid == 0) {
+    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_pair_kernel<GATEUP>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t q = {};
+    q.gridDim = dim3(num_sms());
+    q.blockDim = dim3(kThreads);
+    q.dynamicSmemBytes = C::kSmemBytes;
+    cudaLaunchAttribute ca[1];
+    ca[0].id = cudaLaunchAttributeClusterDimension;
+    ca[0].val.clusterDim.x = 2;
+    ca[0].val.clusterDim.y = 1;
+    ca[0].val.clusterDim.z = 1;
+    q.attrs = ca;
+    q.numAttrs = 1;
+    int clusters = 0;
+    e = cudaOccupancyMaxActiveClusters(&clusters, grouped_gemm_pair_kernel<GATEUP>, &q);
+    if (e != cudaSuccess) return e;
+    if (clusters < 1) return cudaErrorInvalidConfiguration;
+    const int most = num_sms() / 2;
+    grid = 2 * (clusters < most ? clusters : most);
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel<GATEUP>, a0, a1, b16, b128,
+                            args);
+}
+
 // Token tiles of the two expert GEMMs for a batch of T tokens (an expert sees
 // at most T rows, so a small batch gets small tiles and a deeper ring).
 int tile_gateup_for(int64_t T) { return T <= 64 ? 64 : (T <= 1024 ? 128 : 256); }
+
+// Batches with many rows per expert run both expert GEMMs on CTA pairs
+// (256 weight rows per unit, so F and d must be multiples of 256).
+bool use_pairs(const Shape& sh) {
+  return sh.T > 1024 && sh.F % 256 == 0 && sh.d % 256 == 0;
+}
 int tile_down_for(int64_t T) { return T <= 64 ? 64 : (T <= 128 ? 128 : 256); }
 
 // --------------------------------------------------------- CUDA-core path --
@@ -621,7 +950,9 @@ cudaError_t launch_expert_ffn(const Shape& sh, const void* x_perm,
       make_map(&h128, h, rows_cap, (uint64_t)sh.F, 128);
   if (!ok) return cudaErrorInvalidValue;
 
-  const int tgu = tile_gateup_for(sh.T), tdn = tile_down_for(sh.T);
+  const bool pairs = use_pairs(sh);
+  const int tgu = pairs ? 256 : tile_gateup_for(sh.T);
+  const int tdn = pairs ? 256 : tile_down_for(sh.T);
   cudaError_t e = launch_pdl(gemm_plan_kernel, dim3(1), dim3(1024), 0, st, offsets,
                              (int)sh.N, tgu, tdn, tile_start);
   if (e != cudaSuccess) return e;
@@ -638,6 +969,22 @@ cudaError_t launch_expert_ffn(const Shape& sh, const void* x_perm,
   gu.a_rows = gu.out_cols;
   gu.mt_chunk = gu.m_tiles;
   gu.kb_chunk = gu.num_kb;
+  if (pairs) {
+    GemmArgs gp = gu;
+    gp.m_tiles = (int)(sh.F / 256);  // pairs of 128-row tiles
+    e = launch_pair<true>(wg_map, wu_map, x16, x128, gp, st);
+    if (e != cudaSuccess) return e;
+    GemmArgs dp = gu;
+    dp.tile_start = tile_start + sh.N + 1;
+    dp.out = y_perm;
+    dp.num_kb = (int)(sh.F / BK);
+    dp.out_cols = (int)sh.d;
+    dp.a_rows = (int)sh.d;
+    dp.m_tiles = (int)(sh.d / 256);
+    dp.mt_chunk = dp.m_tiles;
+    dp.kb_chunk = dp.num_kb;
+    return launch_pair<false>(wd_map, wd_map, h16, h128, dp, st);
+  }
   e = tgu == 64    ? launch_tc<true, 64>(wg_map, wu_map, x16, x128, gu, st)
       : tgu == 128 ? launch_tc<true, 128>(wg_map, wu_map, x16, x128, gu, st)
                    : launch_tc<true, 256>(wg_map, wu_map, x16, x128, gu, st);

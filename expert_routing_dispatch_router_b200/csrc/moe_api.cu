@@ -269,6 +269,25 @@ moe_status_t moe_layer_forward_host(const moe_config_t* cfg, const void* x_host,
   return MOE_OK;
 }
 
+moe_status_t moe_bias_pid_update(const moe_config_t* cfg, const int32_t* counts,
+                                 float* bias, double* state,
+                                 const moe_pid_params_t* params, moe_stream_t stream) {
+  Shape sh;
+  moe_status_t s = make_shape(cfg, &sh);
+  if (s != MOE_OK) return s;
+  if (!dev_ok(counts) || !dev_ok(bias) || !dev_ok(state) || params == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  const moe_pid_params_t& p = *params;
+  if (!(p.target_routed_share >= 0.f && p.target_routed_share <= 1.f)) return MOE_ERR_INVALID_ARG;
+  const float g[4] = {p.kp, p.ki, p.kd, p.max_step};
+  for (float v : g)
+    if (!isfinite(v) || v < 0.f) return MOE_ERR_INVALID_ARG;
+  if (sh.T == 0) return MOE_OK;
+  return cuda_status(launch_bias_pid(sh, counts, bias, state, p.target_routed_share, p.kp,
+                                     p.ki, p.kd, p.max_step,
+                                     reinterpret_cast<cudaStream_t>(stream)));
+}
+
 moe_status_t moe_read_device_error(void* ws, int32_t* code_out, moe_stream_t stream) {
   if (ws == nullptr) return MOE_ERR_WORKSPACE;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

@@ -84,6 +84,9 @@ int64_t router_planes_rows(const Shape& sh);   // 3E rounded up to 128
 int router_tc_chunks(const Shape& sh);         // contraction chunks of that router
 int router_launch_count(const Shape& sh);
 int expert_ffn_launch_count(const Shape& sh);
+cudaError_t launch_bias_pid(const Shape& sh, const int32_t* counts, float* bias,
+                            double* state, double target, double kp, double ki,
+                            double kd, double max_step, cudaStream_t st);
 int dispatch_launch_count(const Shape& sh);
 bool expert_ffn_uses_tensor_cores(const Shape& sh);
 int num_sms();

@@ -187,6 +187,33 @@ moe_status_t moe_route_noalloc(const moe_config_t* cfg, const void* x,
                                float* topk_gate, uint8_t* flags,
                                moe_stream_t stream);
 
+/* PID controller on the zero experts' router bias, run between layer calls.
+ * "Meituan lancerer LongCat-2.0" (snilld.dk), "MoE i praksis og prisen for
+ * fleksibilitet": a PID controller adjusts the router bias so that the
+ * activated parameters stay in the wanted range. From the per-expert counts of
+ * the last call (moe_layer_forward or moe_dispatch):
+ *   share = sum_{e<N} counts[e] / (T*k)   (slots that ran a routed expert)
+ *   err   = share - target_routed_share
+ *   u     = kp*err + ki*(I + err) + kd*(err - prev), clamped to +-max_step
+ *   bias[e] += u for every zero expert e >= N (routed experts untouched)
+ *   state = {I + err, err}
+ * A share above the target raises the zero experts' keys, so the next call
+ * sends more slots to them. The pages give no gains or set-point.
+ *  counts [E] int32 (device), bias [E] float (device, updated in place),
+ *  state [2] double (device; start from zeros), params on the host.
+ *  cfg->T and top_k must be those of the call that produced counts.
+ *  Returns MOE_ERR_INVALID_ARG for a NULL pointer, a misaligned pointer, a
+ *  target outside [0, 1], or a negative or non-finite gain or max_step. */
+typedef struct {
+  float target_routed_share;
+  float kp, ki, kd;
+  float max_step;
+} moe_pid_params_t;
+
+moe_status_t moe_bias_pid_update(const moe_config_t* cfg, const int32_t* counts,
+                                 float* bias, double* state,
+                                 const moe_pid_params_t* params, moe_stream_t stream);
+
 /* Waits for `stream`, then reads and clears the device-side error word in ws.
  * *code_out (may be NULL) gets 0 when no check failed, else a nonzero code
  * (1 = a bounded wait in the expert GEMM ran out, 2 = a routing slot held an

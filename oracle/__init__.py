@@ -61,6 +61,7 @@ def _load():
                 "oracle_combine": ([I64, I64, I64, I64, D, P, P, P, P, P, P], None),
                 "oracle_layer": ([I64, P, I64, I64, I64, I64, I64, I64, D, I, P, P,
                                   P, P, P, P, P, P, P, P], None),
+                "oracle_pid_update": ([I64, I64, I64, I64, P, P, P, D, D, D, D, D], None),
             }
             for name, (args, res) in sig.items():
                 fn = getattr(lib, name)
@@ -245,3 +246,16 @@ def layer(x, w_router, bias, w_gate, w_up, w_down, n_routed: int, top_k: int,
                          None if fi is None else _p(fi), _p(out), _p(idx),
                          _p(gate))
     return out, idx, gate
+
+
+def pid_update(counts, bias, state, T: int, k: int, n_routed: int, target: float,
+               kp: float, ki: float, kd: float, max_step: float):
+    """One controller step on copies of bias (fp32 [E]) and state (fp64 [2]).
+    Returns (new_bias, new_state)."""
+    c = _i32(counts)
+    b = np.array(_f32(bias), copy=True)
+    st = np.array(_f64(state), copy=True)
+    E = b.shape[0]
+    _load().oracle_pid_update(T, k, n_routed, E, _p(c), _p(b), _p(st), float(target),
+                              float(kp), float(ki), float(kd), float(max_step))
+    return b, st

@@ -350,3 +350,34 @@ void oracle_layer(int64_t n_tok, const int32_t* tokens, int64_t T, int64_t d,
     free(taken);
   }
 }
+
+/* ------------------------------------------------- router bias controller -- */
+
+/* PID update of the zero experts' router bias, reading R13 (see the design
+ * notes): "Meituan lancerer LongCat-2.0" (snilld.dk), "MoE i praksis og
+ * prisen for fleksibilitet", says a PID controller adjusts the router bias so
+ * that the activation stays in the wanted range. The controlled value is the
+ * share of routing slots that went to routed experts,
+ *   share = sum_{e<N} counts[e] / (T k),
+ * the error is err = share - target, and
+ *   u = kp err + ki (I + err) + kd (err - prev)       (I: running sum of err)
+ * clamped to [-max_step, max_step], is added to every zero expert's bias: a
+ * share above target raises the zero experts' keys, so more slots go to them.
+ * state = {I, prev}; both are updated (I += err, prev = err). Routed experts'
+ * biases are left alone. The new bias is rounded to fp32 once. */
+void oracle_pid_update(int64_t T, int64_t k, int64_t N, int64_t E,
+                       const int32_t* counts, float* bias, double* state,
+                       double target, double kp, double ki, double kd,
+                       double max_step) {
+  int64_t routed = 0;
+  for (int64_t e = 0; e < N; ++e) routed += counts[e];
+  const double share = (double)routed / (double)(T * k);
+  const double err = share - target;
+  const double integral = state[0] + err;
+  double u = kp * err + ki * integral + kd * (err - state[1]);
+  if (u > max_step) u = max_step;
+  if (u < -max_step) u = -max_step;
+  for (int64_t e = N; e < E; ++e) bias[e] = (float)((double)bias[e] + u);
+  state[0] = integral;
+  state[1] = err;
+}

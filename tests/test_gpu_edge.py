@@ -70,12 +70,14 @@ def test_all_tokens_to_one_expert_multiple_tiles():
     assert counts[2] == 300
 
 
-@pytest.mark.parametrize("sizes", [(1, 127, 128, 129, 0, 256, 3),
-                                   (255, 0, 0, 1, 17, 384, 64)])
-def test_expert_segments_around_tile_size(sizes):
+@pytest.mark.parametrize("sizes,F", [((1, 127, 128, 129, 0, 256, 3), 384),
+                                     ((255, 0, 0, 1, 17, 384, 64), 384),
+                                     # T > 1024: both GEMMs run on CTA pairs
+                                     ((1, 31, 32, 33, 255, 256, 257, 300), 512)])
+def test_expert_segments_around_tile_size(sizes, F):
     """moe_expert_ffn on crafted segments: offsets give exactly these rows per
     expert; rows are random bf16; checked row by row against the oracle."""
-    N, d, F = len(sizes), 256, 384
+    N, d = len(sizes), 256
     sh = MoEShape("seg", T=sum(sizes), d=d, n_routed=N, n_zero=1, top_k=1, ffn=F)
     inp = make_inputs(sh, 6)
     ls = shape_of(sh)

@@ -34,6 +34,9 @@ SMALL = [
     # skewed: one expert gets most tokens (multiple token tiles per expert)
     MoEShape("skew_bf16", T=517, d=384, n_routed=5, n_zero=3, top_k=2, ffn=256,
              routing="zipf"),
+    # T > 1024 with d, F multiples of 256 -> the expert GEMMs run on CTA pairs
+    MoEShape("pairs_bf16", T=1100, d=512, n_routed=8, n_zero=2, top_k=4, ffn=512,
+             routing="zipf"),
     # d, F not multiples of 128 -> CUDA-core path in bf16
     MoEShape("odd_bf16", T=77, d=200, n_routed=4, n_zero=1, top_k=2, ffn=136),
     CONFIGS["tiny_fp32"],
