@@ -47,7 +47,7 @@ def peaks():
             "source": "fallback"}
 
 
-KERNEL_SOURCES = ("expert_ffn.cu", "sm100_ptx.cuh", "moe_internal.cuh")
+KERNEL_SOURCES = ("expert_ffn.cu", "sm100_ptx.cuh")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "grouped_gemm_tc_traffic.json")
 
 

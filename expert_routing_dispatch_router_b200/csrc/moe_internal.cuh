@@ -26,7 +26,8 @@ constexpr int kErrBadExpertId = 2;
 // Layout of the workspace (byte offsets from its base). Built on the host
 // from the config alone; every region is kWsAlign-aligned.
 struct WsLayout {
-  size_t header;       // int32[64]: [0] error code, [1] error detail
+  size_t header;       // int32[64]: [0] error code, [1] detail, [2..33] router
+                       // group counters (zero between calls)
   size_t logits;       // float router partials: [splits, T, E] or [T, 3E pad]
   size_t planes;       // bf16 [3E pad, d] router weights split in 3 planes
   size_t router_plan;  // int32 [4] plan of the tensor-core router GEMM
@@ -83,6 +84,7 @@ bool router_uses_tensor_cores(const Shape& sh);
 int64_t router_planes_rows(const Shape& sh);   // 3E rounded up to 128
 int router_tc_chunks(const Shape& sh);         // contraction chunks of that router
 int router_launch_count(const Shape& sh);
+int router_small_splits(const Shape& sh);
 int expert_ffn_launch_count(const Shape& sh);
 cudaError_t launch_bias_pid(const Shape& sh, const int32_t* counts, float* bias,
                             double* state, double target, double kp, double ki,

@@ -187,35 +187,19 @@ __device__ __forceinline__ uint32_t ord_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// Top-k of one token by one warp, from its logits lg[i] of experts
+// lane + 32 i: keys = logits + bias, k+1 rounds of a warp arg-max (ties to the
+// lower id), gates = softmax of the selected raw logits, and the near-tie flag.
+// Writes logits_out (if given), idx_out, gate_out and flags (if given) of t.
 template <int PL>
-__global__ void __launch_bounds__(256)
-    topk_kernel(const float* __restrict__ part, int n_outer, int64_t outer_stride,
-                int n_inner, int64_t inner_stride, int64_t row_stride,
-                const float* __restrict__ bias, float* __restrict__ logits_out,
-                int32_t* __restrict__ idx_out, float* __restrict__ gate_out,
-                uint8_t* __restrict__ flags, int64_t T, int E, int k) {
-  griddep_wait();
-  const int lane = threadIdx.x & 31;
-  const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  griddep_launch_dependents();
-  if (t >= T) return;
-
-  // logits = partial sums added in a fixed order (outer, then inner index),
-  // so results are reproducible; the loads of several partials are issued
-  // together
-  float lg[PL], key[PL];
-#pragma unroll
-  for (int i = 0; i < PL; ++i) lg[i] = 0.f;
-  const float* pt = part + t * row_stride + lane;
-  for (int zo = 0; zo < n_outer; ++zo) {
-#pragma unroll 4
-    for (int zi = 0; zi < n_inner; ++zi) {
-      const float* pz = pt + zo * outer_stride + zi * inner_stride;
-#pragma unroll
-      for (int i = 0; i < PL; ++i)
-        if (lane + 32 * i < E) lg[i] += pz[32 * i];
-    }
-  }
+__device__ __forceinline__ void warp_select_token(const float (&lg)[PL],
+                                                  const float* __restrict__ bias,
+                                                  float* __restrict__ logits_out,
+                                                  int32_t* __restrict__ idx_out,
+                                                  float* __restrict__ gate_out,
+                                                  uint8_t* __restrict__ flags, int64_t t,
+                                                  int E, int k, int lane) {
+  float key[PL];
 #pragma unroll
   for (int i = 0; i < PL; ++i) {
     const int e = lane + 32 * i;
@@ -288,6 +272,39 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+
+template <int PL>
+__global__ void __launch_bounds__(256)
+    topk_kernel(const float* __restrict__ part, int n_outer, int64_t outer_stride,
+                int n_inner, int64_t inner_stride, int64_t row_stride,
+                const float* __restrict__ bias, float* __restrict__ logits_out,
+                int32_t* __restrict__ idx_out, float* __restrict__ gate_out,
+                uint8_t* __restrict__ flags, int64_t T, int E, int k) {
+  griddep_wait();
+  const int lane = threadIdx.x & 31;
+  const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  griddep_launch_dependents();
+  if (t >= T) return;
+
+  // logits = partial sums added in a fixed order (outer, then inner index),
+  // so results are reproducible; the loads of several partials are issued
+  // together
+  float lg[PL];
+#pragma unroll
+  for (int i = 0; i < PL; ++i) lg[i] = 0.f;
+  const float* pt = part + t * row_stride + lane;
+  for (int zo = 0; zo < n_outer; ++zo) {
+#pragma unroll 4
+    for (int zi = 0; zi < n_inner; ++zi) {
+      const float* pz = pt + zo * outer_stride + zi * inner_stride;
+#pragma unroll
+      for (int i = 0; i < PL; ++i)
+        if (lane + 32 * i < E) lg[i] += pz[32 * i];
+    }
+  }
+  warp_select_token<PL>(lg, bias, logits_out, idx_out, gate_out, flags, t, E, k, lane);
+}
+
 template <int PL>
 void launch_topk(const float* part, int n_outer, int64_t outer_stride, int n_inner,
                  int64_t inner_stride, int64_t row_stride, const float* bias,
@@ -298,6 +315,124 @@ void launch_topk(const float* part, int n_outer, int64_t outer_stride, int n_inn
   launch_pdl(topk_kernel<PL>, dim3(grid), dim3(warps * 32), 0, st, part, n_outer,
              outer_stride, n_inner, inner_stride, row_stride, bias,
              logits, idx, gate, flags, T, E, k);
+}
+
+// ------------------------------------------------------- small batches --
+// Router for T <= 256 in one launch. CTA (g, et, z) takes the 8 tokens of
+// group g, the 32 experts of tile et and contraction split z (<= 1024
+// elements). Its x rows sit in shared memory as fp32; each warp streams 4
+// router rows from global memory, lanes along the contraction (coalesced).
+// A lane sums its 32-element share, a warp tree adds the lanes, and the
+// partial sums of the splits go to the workspace. The last CTA to finish a
+// token group (a counter per group, incremented after a fence) adds the
+// partials of its 8 tokens in split order and runs their top-k, then resets
+// the counter to zero for the next call. No CTA waits for another.
+constexpr int DG = 8;    // tokens per group
+constexpr int DE = 32;   // experts per CTA (8 warps x 4)
+
+template <typename XT>
+__device__ __forceinline__ void load_x8(const XT* x, int64_t off, float* dst);
+template <>
+__device__ __forceinline__ void load_x8<__nv_bfloat16>(const __nv_bfloat16* x, int64_t off,
+                                                       float* dst) {
+  const uint4 v = *reinterpret_cast<const uint4*>(x + off);
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    dst[2 * i] = __uint_as_float(w[i] << 16);
+    dst[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+template <>
+__device__ __forceinline__ void load_x8<float>(const float* x, int64_t off, float* dst) {
+  const float4 a = *reinterpret_cast<const float4*>(x + off);
+  const float4 b = *reinterpret_cast<const float4*>(x + off + 4);
+  dst[0] = a.x; dst[1] = a.y; dst[2] = a.z; dst[3] = a.w;
+  dst[4] = b.x; dst[5] = b.y; dst[6] = b.z; dst[7] = b.w;
+}
+
+template <typename XT, int PL>
+__global__ void __launch_bounds__(256)
+    router_small_kernel(const XT* __restrict__ x, const float* __restrict__ w_r,
+                        const float* __restrict__ bias, float* __restrict__ part,
+                        int32_t* __restrict__ counter, float* __restrict__ logits_out,
+                        int32_t* __restrict__ idx_out, float* __restrict__ gate_out,
+                        uint8_t* __restrict__ flags, int64_t T, int64_t d, int E, int k,
+                        int64_t ksplit) {
+  extern __shared__ float xs[];  // [DG][ksplit]
+  __shared__ int s_last;
+  griddep_wait();
+  griddep_launch_dependents();
+  const int g = blockIdx.x, et = blockIdx.y, z = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t t0 = (int64_t)g * DG;
+  const int64_t kbeg = (int64_t)z * ksplit;
+  const int64_t klen = min(d, kbeg + ksplit) - kbeg;
+  const int64_t v8 = klen / 8;
+  for (int64_t i = threadIdx.x; i < DG * v8; i += blockDim.x) {
+    const int tt = (int)(i / v8);
+    const int64_t kk = (i - tt * v8) * 8;
+    float* dst = xs + tt * ksplit + kk;
+    if (t0 + tt < T) {
+      load_x8<XT>(x, (t0 + tt) * d + kbeg + kk, dst);
+    } else {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) dst[q] = 0.f;
+    }
+  }
+  __syncthreads();
+  for (int j = 0; j < 4; ++j) {
+    const int e = et * DE + warp * 4 + j;
+    if (e >= E) break;
+    const float* wr = w_r + (int64_t)e * d + kbeg;
+    float acc[DG];
+#pragma unroll
+    for (int tt = 0; tt < DG; ++tt) acc[tt] = 0.f;
+    for (int64_t kk = 4 * lane; kk < klen; kk += 128) {
+      const float4 wv = *reinterpret_cast<const float4*>(wr + kk);
+#pragma unroll
+      for (int tt = 0; tt < DG; ++tt) {
+        const float4 xv = *reinterpret_cast<const float4*>(xs + tt * ksplit + kk);
+        acc[tt] = fmaf(wv.x, xv.x, acc[tt]);
+        acc[tt] = fmaf(wv.y, xv.y, acc[tt]);
+        acc[tt] = fmaf(wv.z, xv.z, acc[tt]);
+        acc[tt] = fmaf(wv.w, xv.w, acc[tt]);
+      }
+    }
+#pragma unroll
+    for (int tt = 0; tt < DG; ++tt)
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1)
+        acc[tt] += __shfl_xor_sync(0xffffffffu, acc[tt], off);
+    if (lane < DG && t0 + lane < T) {
+      float v = acc[0];
+#pragma unroll
+      for (int tt = 1; tt < DG; ++tt)
+        if (lane == tt) v = acc[tt];
+      part[((int64_t)z * T + t0 + lane) * E + e] = v;
+    }
+  }
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0)
+    s_last = atomicAdd(&counter[g], 1) == (int)(gridDim.y * gridDim.z) - 1;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  const int64_t t = t0 + warp;
+  if (t < T) {
+    float lg[PL];
+#pragma unroll
+    for (int i = 0; i < PL; ++i) lg[i] = 0.f;
+    for (int zz = 0; zz < (int)gridDim.z; ++zz) {
+      const float* pz = part + ((int64_t)zz * T + t) * E + lane;
+#pragma unroll
+      for (int i = 0; i < PL; ++i)
+        if (lane + 32 * i < E) lg[i] += __ldcg(pz + 32 * i);
+    }
+    warp_select_token<PL>(lg, bias, logits_out, idx_out, gate_out, flags, t, E, k, lane);
+  }
+  if (threadIdx.x == 0) counter[g] = 0;
 }
 
 // Exact three-way split of the fp32 router weights into bf16 planes for the
@@ -374,7 +509,16 @@ bool router_uses_tensor_cores(const Shape& sh) {
          router_planes_rows(sh) <= 4096;
 }
 
-int router_launch_count(const Shape& sh) { return router_uses_tensor_cores(sh) ? 3 : 2; }
+constexpr int64_t kSmallRouterMaxTokens = 256;
+
+bool router_uses_small_kernel(const Shape& sh) { return sh.T <= kSmallRouterMaxTokens; }
+
+// Contraction splits of the small-batch router (<= 1024 elements each).
+int router_small_splits(const Shape& sh) { return (int)((sh.d + 1023) / 1024); }
+
+int router_launch_count(const Shape& sh) {
+  return router_uses_tensor_cores(sh) ? 3 : (router_uses_small_kernel(sh) ? 1 : 2);
+}
 
 // Number of contraction splits so that the logits GEMM has >= ~2 CTAs per SM.
 int router_splits(const Shape& sh) {
@@ -395,6 +539,34 @@ cudaError_t launch_router(const Shape& sh, const void* x, const float* w_r,
   int n_outer, n_inner;
   int64_t outer_stride, inner_stride, row_stride;
   cudaError_t e;
+  if (router_uses_small_kernel(sh)) {
+    // one launch: logits, split sums and top-k; the group counters live in
+    // the workspace header after the error word (zero between calls)
+    const int nsplit = router_small_splits(sh);
+    int64_t ksplit = (sh.d + nsplit - 1) / nsplit;
+    ksplit = (ksplit + 7) / 8 * 8;
+    const dim3 grid((unsigned)((sh.T + DG - 1) / DG), (unsigned)((sh.E + DE - 1) / DE),
+                    (unsigned)nsplit);
+    const size_t smem = (size_t)DG * ksplit * sizeof(float);
+    int32_t* counter = err + 2;
+    const int pl = (int)((sh.E + 31) / 32);
+    const int E = (int)sh.E, k = (int)sh.k;
+#define MOE_SMALL(XT, P)                                                              \
+  launch_pdl(router_small_kernel<XT, P>, grid, dim3(256), smem, st,                   \
+             static_cast<const XT*>(x), w_r, bias, part, counter, logits_out, idx, gate, \
+             flags, sh.T, sh.d, E, k, ksplit)
+#define MOE_SMALL_PL(XT)                    \
+  (pl <= 1    ? MOE_SMALL(XT, 1)            \
+   : pl <= 2  ? MOE_SMALL(XT, 2)            \
+   : pl <= 4  ? MOE_SMALL(XT, 4)            \
+   : pl <= 8  ? MOE_SMALL(XT, 8)            \
+   : pl <= 16 ? MOE_SMALL(XT, 16)           \
+              : MOE_SMALL(XT, 32))
+    e = sh.bf16 ? MOE_SMALL_PL(__nv_bfloat16) : MOE_SMALL_PL(float);
+#undef MOE_SMALL_PL
+#undef MOE_SMALL
+    return e;
+  }
   if (router_uses_tensor_cores(sh)) {
     const int64_t Ep = router_planes_rows(sh);
     const int64_t n4 = sh.E * sh.d / 4;

@@ -45,8 +45,9 @@
  *  - Workspace: every call that takes `ws` needs ws_bytes >=
  *    moe_workspace_size(cfg) and a 256-byte aligned `ws`; the same workspace
  *    serves all calls of one config. Its first 256 bytes hold the device
- *    error word and must be zero before first use (cudaMemset once);
- *    moe_read_device_error clears it again. Calls that share a workspace must
+ *    error word and small counters that the kernels return to zero; they
+ *    must be zero before first use (cudaMemset once). moe_read_device_error
+ *    clears the error word again. Calls that share a workspace must
  *    be ordered on one stream.
  */
 #ifndef MOE_API_H
