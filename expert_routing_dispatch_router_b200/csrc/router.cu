@@ -327,6 +327,31 @@ void launch_topk(const float* part, int n_outer, int64_t outer_stride, int n_inn
 // token group (a counter per group, incremented after a fence) adds the
 // partials of its 8 tokens in split order and runs their top-k, then resets
 // the counter to zero for the next call. No CTA waits for another.
+//
+// Weight prefetch (the fused layer call at T <= 64): while the router and
+// dispatch run, HBM would sit idle, so the router's CTAs first ask L2 to fetch
+// the weight tiles the gate/up GEMM reads first. At T <= 64 every touched
+// expert is one token tile, and the GEMM's units run expert by expert, so
+// unit u is (expert u / m_tiles, rows (u % m_tiles) * 128) when every expert is
+// touched; the first pf_units such tiles of W_gate and W_up are requested.
+// This only moves bytes earlier; a wrong guess costs idle bandwidth.
+struct WeightPrefetch {
+  const uint8_t* w_gate = nullptr;  // [N, F, d] bf16, or null for none
+  const uint8_t* w_up = nullptr;
+  int64_t expert_bytes = 0;  // F * d * 2
+  int64_t tile_bytes = 0;    // 128 rows * d * 2 (contiguous)
+  int m_tiles = 0;           // F / 128
+  int units = 0;             // tiles of each matrix to request
+};
+// Bring `bytes` (16-byte aligned, a multiple of 16) of global memory into L2,
+// asynchronously; nothing waits for it.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(
+                   reinterpret_cast<uint64_t>(p)),
+               "r"(bytes)
+               : "memory");
+}
+
 constexpr int DG = 8;    // tokens per group
 constexpr int DE = 32;   // experts per CTA (8 warps x 4)
 
@@ -351,18 +376,31 @@ __device__ __forceinline__ void load_x8<float>(const float* x, int64_t off, floa
   dst[4] = b.x; dst[5] = b.y; dst[6] = b.z; dst[7] = b.w;
 }
 
-template <typename XT, int PL>
+// ITER: 128-element steps per lane in one split (ksplit = 128 * ITER), a
+// compile-time count so that all of a warp's router-row loads are in flight
+// together instead of one round trip per step.
+template <typename XT, int PL, int ITER>
 __global__ void __launch_bounds__(256)
     router_small_kernel(const XT* __restrict__ x, const float* __restrict__ w_r,
                         const float* __restrict__ bias, float* __restrict__ part,
                         int32_t* __restrict__ counter, float* __restrict__ logits_out,
                         int32_t* __restrict__ idx_out, float* __restrict__ gate_out,
                         uint8_t* __restrict__ flags, int64_t T, int64_t d, int E, int k,
-                        int64_t ksplit) {
+                        int64_t ksplit, const WeightPrefetch pf) {
   extern __shared__ float xs[];  // [DG][ksplit]
   __shared__ int s_last;
   griddep_wait();
   griddep_launch_dependents();
+  if (pf.units > 0 && threadIdx.x == 0) {
+    const int nctas = gridDim.x * gridDim.y * gridDim.z;
+    const int c = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
+    for (int u = c; u < pf.units; u += nctas) {
+      const int64_t off = (int64_t)(u / pf.m_tiles) * pf.expert_bytes +
+                          (int64_t)(u % pf.m_tiles) * pf.tile_bytes;
+      prefetch_l2_bulk(pf.w_gate + off, (uint32_t)pf.tile_bytes);
+      prefetch_l2_bulk(pf.w_up + off, (uint32_t)pf.tile_bytes);
+    }
+  }
   const int g = blockIdx.x, et = blockIdx.y, z = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t t0 = (int64_t)g * DG;
@@ -381,22 +419,38 @@ __global__ void __launch_bounds__(256)
     }
   }
   __syncthreads();
+  // the 4 experts of this warp: all their router-row loads first
+  float4 wv[4][ITER];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int e = et * DE + warp * 4 + j;
+    const float* wr = w_r + (int64_t)e * d + kbeg;
+#pragma unroll
+    for (int it = 0; it < ITER; ++it) {
+      const int64_t kk = 4 * lane + 128 * it;
+      wv[j][it] = (e < E && kk < klen) ? *reinterpret_cast<const float4*>(wr + kk)
+                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
+#pragma unroll
   for (int j = 0; j < 4; ++j) {
     const int e = et * DE + warp * 4 + j;
     if (e >= E) break;
-    const float* wr = w_r + (int64_t)e * d + kbeg;
     float acc[DG];
 #pragma unroll
     for (int tt = 0; tt < DG; ++tt) acc[tt] = 0.f;
-    for (int64_t kk = 4 * lane; kk < klen; kk += 128) {
-      const float4 wv = *reinterpret_cast<const float4*>(wr + kk);
+#pragma unroll
+    for (int it = 0; it < ITER; ++it) {
+      const int64_t kk = 4 * lane + 128 * it;
+      if (kk >= klen) break;
+      const float4 w4 = wv[j][it];
 #pragma unroll
       for (int tt = 0; tt < DG; ++tt) {
         const float4 xv = *reinterpret_cast<const float4*>(xs + tt * ksplit + kk);
-        acc[tt] = fmaf(wv.x, xv.x, acc[tt]);
-        acc[tt] = fmaf(wv.y, xv.y, acc[tt]);
-        acc[tt] = fmaf(wv.z, xv.z, acc[tt]);
-        acc[tt] = fmaf(wv.w, xv.w, acc[tt]);
+        acc[tt] = fmaf(w4.x, xv.x, acc[tt]);
+        acc[tt] = fmaf(w4.y, xv.y, acc[tt]);
+        acc[tt] = fmaf(w4.z, xv.z, acc[tt]);
+        acc[tt] = fmaf(w4.w, xv.w, acc[tt]);
       }
     }
 #pragma unroll
@@ -510,6 +564,7 @@ bool router_uses_tensor_cores(const Shape& sh) {
 }
 
 constexpr int64_t kSmallRouterMaxTokens = 256;
+constexpr int64_t kPrefetchBytes = 96ll << 20;  // L2 prefetch budget of a decode call
 
 bool router_uses_small_kernel(const Shape& sh) { return sh.T <= kSmallRouterMaxTokens; }
 
@@ -535,6 +590,7 @@ cudaError_t launch_router(const Shape& sh, const void* x, const float* w_r,
                           const float* bias, float* part, int32_t* idx,
                           float* gate, uint8_t* flags, float* logits_out,
                           void* planes, int32_t* plan, int32_t* err,
+                          const void* prefetch_gate, const void* prefetch_up,
                           cudaStream_t st) {
   int n_outer, n_inner;
   int64_t outer_stride, inner_stride, row_stride;
@@ -543,18 +599,37 @@ cudaError_t launch_router(const Shape& sh, const void* x, const float* w_r,
     // one launch: logits, split sums and top-k; the group counters live in
     // the workspace header after the error word (zero between calls)
     const int nsplit = router_small_splits(sh);
-    int64_t ksplit = (sh.d + nsplit - 1) / nsplit;
-    ksplit = (ksplit + 7) / 8 * 8;
+    const int64_t steps = ((sh.d + nsplit - 1) / nsplit + 127) / 128;  // <= 8
+    const int iter = steps <= 1 ? 1 : steps <= 2 ? 2 : steps <= 4 ? 4 : 8;
+    const int64_t ksplit = 128 * (int64_t)iter;
     const dim3 grid((unsigned)((sh.T + DG - 1) / DG), (unsigned)((sh.E + DE - 1) / DE),
                     (unsigned)nsplit);
     const size_t smem = (size_t)DG * ksplit * sizeof(float);
     int32_t* counter = err + 2;
+    WeightPrefetch pf;
+    const bool aligned = ((reinterpret_cast<uintptr_t>(prefetch_gate) |
+                           reinterpret_cast<uintptr_t>(prefetch_up)) & 15) == 0;
+    if (prefetch_gate && prefetch_up && aligned && sh.T <= 64 && sh.N > 0 &&
+        expert_ffn_uses_tensor_cores(sh)) {
+      pf.w_gate = static_cast<const uint8_t*>(prefetch_gate);
+      pf.w_up = static_cast<const uint8_t*>(prefetch_up);
+      pf.expert_bytes = sh.F * sh.d * 2;
+      pf.tile_bytes = 128 * sh.d * 2;
+      pf.m_tiles = (int)(sh.F / 128);
+      const int64_t budget = kPrefetchBytes / (2 * pf.tile_bytes);  // tiles per matrix
+      const int64_t all = sh.N * pf.m_tiles;
+      pf.units = (int)(budget < all ? budget : all);
+    }
     const int pl = (int)((sh.E + 31) / 32);
     const int E = (int)sh.E, k = (int)sh.k;
-#define MOE_SMALL(XT, P)                                                              \
-  launch_pdl(router_small_kernel<XT, P>, grid, dim3(256), smem, st,                   \
+#define MOE_SMALL_IT(XT, P, I)                                                        \
+  launch_pdl(router_small_kernel<XT, P, I>, grid, dim3(256), smem, st,                \
              static_cast<const XT*>(x), w_r, bias, part, counter, logits_out, idx, gate, \
-             flags, sh.T, sh.d, E, k, ksplit)
+             flags, sh.T, sh.d, E, k, ksplit, pf)
+#define MOE_SMALL(XT, P)                                          \
+  (iter == 1 ? MOE_SMALL_IT(XT, P, 1)                             \
+   : iter == 2 ? MOE_SMALL_IT(XT, P, 2)                           \
+   : iter == 4 ? MOE_SMALL_IT(XT, P, 4) : MOE_SMALL_IT(XT, P, 8))
 #define MOE_SMALL_PL(XT)                    \
   (pl <= 1    ? MOE_SMALL(XT, 1)            \
    : pl <= 2  ? MOE_SMALL(XT, 2)            \
@@ -565,6 +640,7 @@ cudaError_t launch_router(const Shape& sh, const void* x, const float* w_r,
     e = sh.bf16 ? MOE_SMALL_PL(__nv_bfloat16) : MOE_SMALL_PL(float);
 #undef MOE_SMALL_PL
 #undef MOE_SMALL
+#undef MOE_SMALL_IT
     return e;
   }
   if (router_uses_tensor_cores(sh)) {
