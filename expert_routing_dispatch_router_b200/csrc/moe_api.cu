@@ -117,7 +117,7 @@ moe_status_t run_layer(const Shape& sh, const void* x, const float* w_router,
   void* y_perm = at<void>(ws, L.y_perm);
   cudaError_t e = launch_router(sh, x, w_router, bias, at<float>(ws, L.logits), idx,
                                 gate, nullptr, nullptr, at<void>(ws, L.planes),
-                                at<int32_t>(ws, L.router_plan), err, w_gate, w_up, st);
+                                at<int32_t>(ws, L.router_plan), err, st);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   e = launch_dispatch(sh, x, idx, at<int32_t>(ws, L.chunk_base),
                       counts ? counts : at<int32_t>(ws, L.counts), offsets,
@@ -161,7 +161,7 @@ moe_status_t moe_route(const moe_config_t* cfg, const void* x, const float* w_ro
   return cuda_status(launch_router(sh, x, w_router, bias, at<float>(ws, L.logits),
                                    topk_idx, topk_gate, flags, logits,
                                    at<void>(ws, L.planes), at<int32_t>(ws, L.router_plan),
-                                   at<int32_t>(ws, L.header), nullptr, nullptr,
+                                   at<int32_t>(ws, L.header),
                                    reinterpret_cast<cudaStream_t>(stream)));
 }
 

@@ -63,7 +63,6 @@ cudaError_t launch_router(const Shape& sh, const void* x, const float* w_r,
                           const float* bias, float* part, int32_t* idx,
                           float* gate, uint8_t* flags, float* logits_out,
                           void* planes, int32_t* plan, int32_t* err,
-                          const void* prefetch_gate, const void* prefetch_up,
                           cudaStream_t st);
 cudaError_t launch_dispatch(const Shape& sh, const void* x, const int32_t* idx,
                             int32_t* chunk_base, int32_t* counts,

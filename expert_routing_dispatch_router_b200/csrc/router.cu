@@ -18,10 +18,15 @@
 // ceil(E/32) per lane. k+1 rounds of a warp arg-max (ties to the lower id)
 // give the selection in descending key order and the margin between the k-th
 // and (k+1)-th key.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <float.h>
 #include <math.h>
 
+#include <atomic>
+
 #include "moe_internal.cuh"
+#include "sm100_ptx.cuh"
 
 namespace moe {
 namespace {
@@ -187,69 +192,104 @@ __device__ __forceinline__ uint32_t ord_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// Correction bias of experts lane + 32 i (0 past E), loaded ahead of the
+// selection so that its latency overlaps other work.
+template <int PL>
+__device__ __forceinline__ void load_bias(const float* __restrict__ bias, int E, int lane,
+                                          float (&bv)[PL]) {
+#pragma unroll
+  for (int i = 0; i < PL; ++i) bv[i] = (lane + 32 * i < E) ? bias[lane + 32 * i] : 0.f;
+}
+
+__device__ __forceinline__ float ord_key_inv(uint32_t o) {
+  return __uint_as_float((o & 0x80000000u) ? (o & 0x7fffffffu) : ~o);
+}
+
+// Sorts a lane's (key, id) pairs so that larger keys come first and, among
+// equal keys, lower ids (a bitonic network; N is a power of two).
+template <int N>
+__device__ __forceinline__ void sort_pairs_desc(uint32_t (&o)[N], int (&id)[N]) {
+#pragma unroll
+  for (int size = 2; size <= N; size <<= 1)
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1)
+#pragma unroll
+      for (int i = 0; i < N; ++i) {
+        const int j = i ^ stride;
+        if (j > i) {
+          const bool i_first = o[i] > o[j] || (o[i] == o[j] && id[i] < id[j]);
+          const bool swap = ((i & size) == 0) ? !i_first : i_first;
+          const uint32_t oi = o[i], oj = o[j];
+          const int di = id[i], dj = id[j];
+          o[i] = swap ? oj : oi;
+          o[j] = swap ? oi : oj;
+          id[i] = swap ? dj : di;
+          id[j] = swap ? di : dj;
+        }
+      }
+}
+
 // Top-k of one token by one warp, from its logits lg[i] of experts
 // lane + 32 i: keys = logits + bias, k+1 rounds of a warp arg-max (ties to the
 // lower id), gates = softmax of the selected raw logits, and the near-tie flag.
-// Writes logits_out (if given), idx_out, gate_out and flags (if given) of t.
+// Each lane first sorts its own keys, so a round is two warp reductions over
+// the lanes' heads: the largest key, then the lowest id holding it; the
+// winning lane drops its head. Writes logits_out (if given), idx_out,
+// gate_out and flags (if given) of t.
 template <int PL>
 __device__ __forceinline__ void warp_select_token(const float (&lg)[PL],
-                                                  const float* __restrict__ bias,
+                                                  const float (&bv)[PL],
                                                   float* __restrict__ logits_out,
                                                   int32_t* __restrict__ idx_out,
                                                   float* __restrict__ gate_out,
                                                   uint8_t* __restrict__ flags, int64_t t,
                                                   int E, int k, int lane) {
-  float key[PL];
+  // ordered keys: a NaN key counts as -inf; 0 marks an empty slot, below the
+  // key of -inf
+  uint32_t o[PL];
+  int id[PL];
 #pragma unroll
   for (int i = 0; i < PL; ++i) {
     const int e = lane + 32 * i;
-    key[i] = -INFINITY;
+    o[i] = 0u;
+    id[i] = 0x7fffffff;
     if (e < E) {
-      const float kv = lg[i] + bias[e];
-      key[i] = (kv != kv) ? -INFINITY : kv;  // a NaN key never wins
+      const float kv = lg[i] + bv[i];
+      o[i] = ord_key((kv != kv) ? -INFINITY : kv);
+      id[i] = e;
       if (logits_out) logits_out[t * E + e] = lg[i];
     }
   }
+  sort_pairs_desc<PL>(o, id);
 
-  // Each round: every lane takes its best remaining key (ascending ids, so the
-  // lower id wins ties), then two warp reductions pick the largest key and,
-  // among lanes holding it, the lowest id.
-  uint32_t taken = 0;  // bit i: expert lane + 32 i already selected
-  float kth_key = 0.f, next_key = -INFINITY;
-  float my_logit = 0.f;
+  uint32_t kth_o = 0u, next_o = 0u;
   int my_e = 0;
-  const int rounds = (k < E) ? k + 1 : k;
+  const int rounds = (k < E) ? k + 1 : k;  // never more than the E real keys
   for (int j = 0; j < rounds; ++j) {
-    uint32_t bo = 0u;
-    int be = 0x7fffffff;
-    float bk = -INFINITY, bl = 0.f;
+    const uint32_t mo = __reduce_max_sync(0xffffffffu, o[0]);
+    const uint32_t we = __reduce_min_sync(0xffffffffu, o[0] == mo ? (uint32_t)id[0] : 0xffffffffu);
+    if (lane == (int)(we & 31u)) {
 #pragma unroll
-    for (int i = 0; i < PL; ++i) {
-      const int e = lane + 32 * i;
-      const uint32_t o = ord_key(key[i]);
-      if (e < E && !((taken >> i) & 1u) && (be == 0x7fffffff || o > bo)) {
-        bo = o;
-        be = e;
-        bk = key[i];
-        bl = lg[i];
+      for (int i = 0; i + 1 < PL; ++i) {
+        o[i] = o[i + 1];
+        id[i] = id[i + 1];
       }
+      o[PL - 1] = 0u;
+      id[PL - 1] = 0x7fffffff;
     }
-    const uint32_t mo = __reduce_max_sync(0xffffffffu, bo);
-    const int we = (int)__reduce_min_sync(0xffffffffu,
-                                          (be != 0x7fffffff && bo == mo) ? (uint32_t)be
-                                                                        : 0x7fffffffu);
-    const float wk = __shfl_sync(0xffffffffu, bk, we & 31);
-    const float wl = __shfl_sync(0xffffffffu, bl, we & 31);
     if (j < k) {
-      if (lane == (we & 31)) taken |= 1u << (we >> 5);
-      if (lane == j) {
-        my_logit = wl;
-        my_e = we;
-      }
-      kth_key = wk;
+      if (lane == j) my_e = (int)we;
+      kth_o = mo;
     } else {
-      next_key = wk;
+      next_o = mo;
     }
+  }
+  // raw logit of this lane's pick, from the lane that holds it
+  float my_logit = 0.f;
+#pragma unroll
+  for (int i = 0; i < PL; ++i) {
+    const float v = __shfl_sync(0xffffffffu, lg[i], my_e & 31);
+    if ((my_e >> 5) == i) my_logit = v;
   }
 
   // gates: softmax of the selected raw logits
@@ -267,7 +307,7 @@ __device__ __forceinline__ void warp_select_token(const float (&lg)[PL],
     gate_out[t * k + lane] = p / zsum;
   }
   if (flags && lane == 0) {
-    const float margin = (k < E) ? kth_key - next_key : INFINITY;
+    const float margin = (k < E) ? ord_key_inv(kth_o) - ord_key_inv(next_o) : INFINITY;
     flags[t] = (margin < 1e-4f) ? 1 : 0;
   }
 }
@@ -285,6 +325,8 @@ __global__ void __launch_bounds__(256)
   const int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   griddep_launch_dependents();
   if (t >= T) return;
+  float bv[PL];
+  load_bias<PL>(bias, E, lane, bv);
 
   // logits = partial sums added in a fixed order (outer, then inner index),
   // so results are reproducible; the loads of several partials are issued
@@ -302,7 +344,7 @@ __global__ void __launch_bounds__(256)
         if (lane + 32 * i < E) lg[i] += pz[32 * i];
     }
   }
-  warp_select_token<PL>(lg, bias, logits_out, idx_out, gate_out, flags, t, E, k, lane);
+  warp_select_token<PL>(lg, bv, logits_out, idx_out, gate_out, flags, t, E, k, lane);
 }
 
 template <int PL>
@@ -319,172 +361,212 @@ void launch_topk(const float* part, int n_outer, int64_t outer_stride, int n_inn
 
 // ------------------------------------------------------- small batches --
 // Router for T <= 256 in one launch. CTA (g, et, z) takes the 8 tokens of
-// group g, the 32 experts of tile et and contraction split z (<= 1024
-// elements). Its x rows sit in shared memory as fp32; each warp streams 4
-// router rows from global memory, lanes along the contraction (coalesced).
-// A lane sums its 32-element share, a warp tree adds the lanes, and the
-// partial sums of the splits go to the workspace. The last CTA to finish a
-// token group (a counter per group, incremented after a fence) adds the
-// partials of its 8 tokens in split order and runs their top-k, then resets
-// the counter to zero for the next call. No CTA waits for another.
-//
-// Weight prefetch (the fused layer call at T <= 64): while the router and
-// dispatch run, HBM would sit idle, so the router's CTAs first ask L2 to fetch
-// the weight tiles the gate/up GEMM reads first. At T <= 64 every touched
-// expert is one token tile, and the GEMM's units run expert by expert, so
-// unit u is (expert u / m_tiles, rows (u % m_tiles) * 128) when every expert is
-// touched; the first pf_units such tiles of W_gate and W_up are requested.
-// This only moves bytes earlier; a wrong guess costs idle bandwidth.
-struct WeightPrefetch {
-  const uint8_t* w_gate = nullptr;  // [N, F, d] bf16, or null for none
-  const uint8_t* w_up = nullptr;
-  int64_t expert_bytes = 0;  // F * d * 2
-  int64_t tile_bytes = 0;    // 128 rows * d * 2 (contiguous)
-  int m_tiles = 0;           // F / 128
-  int units = 0;             // tiles of each matrix to request
-};
-// Bring `bytes` (16-byte aligned, a multiple of 16) of global memory into L2,
-// asynchronously; nothing waits for it.
-__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(
-                   reinterpret_cast<uint64_t>(p)),
-               "r"(bytes)
-               : "memory");
-}
+// group g, the 32 experts of tile et and the contraction range
+// [z * ksplit, (z + 1) * ksplit). The host picks ksplit (a multiple of 32) so
+// that the grid fills the SMs once where shared memory allows. One thread
+// brings the CTA's router rows (a 32 x 256 box) and x rows (an 8 x 256 box)
+// into shared memory by TMA, chunk by chunk, one mbarrier per chunk, so the
+// arithmetic on a chunk starts as soon as that chunk has landed; rows past E
+// or T and columns past d arrive as zeros. Each warp
+// computes 4 experts x 8 tokens with lanes along the contraction; a warp tree
+// adds the lanes, and the partial sums of the splits go to the workspace. The
+// last CTA to finish a token group (a counter per group, incremented after a
+// fence) adds the partials of its 8 tokens in split order and runs their
+// top-k, then resets the counter to zero for the next call. No CTA waits for
+// another. A chunk that has not landed within the wait limit sets the error
+// word; the CTA still takes its turn on the counter, so the counters stay
+// consistent.
+constexpr int DG = 8;             // tokens per group
+constexpr int DE = 32;            // experts per CTA (8 warps x 4)
+constexpr int kSmallChunk = 256;  // contraction elements per mbarrier
+constexpr int kSmallHeader = 128; // shared bytes before the first chunk
+constexpr int kSmallMaxBytes = 220 * 1024;  // shared memory budget of one CTA
+constexpr int kSmallMaxChunks = (kSmallHeader - 16) / 8;
+constexpr uint64_t kSmallWaitNs = 2000000000ull;  // wait limit for a chunk
 
-constexpr int DG = 8;    // tokens per group
-constexpr int DE = 32;   // experts per CTA (8 warps x 4)
-
-template <typename XT>
-__device__ __forceinline__ void load_x8(const XT* x, int64_t off, float* dst);
-template <>
-__device__ __forceinline__ void load_x8<__nv_bfloat16>(const __nv_bfloat16* x, int64_t off,
-                                                       float* dst) {
-  const uint4 v = *reinterpret_cast<const uint4*>(x + off);
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    dst[2 * i] = __uint_as_float(w[i] << 16);
-    dst[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-  }
-}
-template <>
-__device__ __forceinline__ void load_x8<float>(const float* x, int64_t off, float* dst) {
-  const float4 a = *reinterpret_cast<const float4*>(x + off);
-  const float4 b = *reinterpret_cast<const float4*>(x + off + 4);
-  dst[0] = a.x; dst[1] = a.y; dst[2] = a.z; dst[3] = a.w;
-  dst[4] = b.x; dst[5] = b.y; dst[6] = b.z; dst[7] = b.w;
-}
-
-// ITER: 128-element steps per lane in one split (ksplit = 128 * ITER), a
-// compile-time count so that all of a warp's router-row loads are in flight
-// together instead of one round trip per step.
-template <typename XT, int PL, int ITER>
-__global__ void __launch_bounds__(256)
-    router_small_kernel(const XT* __restrict__ x, const float* __restrict__ w_r,
-                        const float* __restrict__ bias, float* __restrict__ part,
-                        int32_t* __restrict__ counter, float* __restrict__ logits_out,
-                        int32_t* __restrict__ idx_out, float* __restrict__ gate_out,
-                        uint8_t* __restrict__ flags, int64_t T, int64_t d, int E, int k,
-                        int64_t ksplit, const WeightPrefetch pf) {
-  extern __shared__ float xs[];  // [DG][ksplit]
-  __shared__ int s_last;
-  griddep_wait();
-  griddep_launch_dependents();
-  if (pf.units > 0 && threadIdx.x == 0) {
-    const int nctas = gridDim.x * gridDim.y * gridDim.z;
-    const int c = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
-    for (int u = c; u < pf.units; u += nctas) {
-      const int64_t off = (int64_t)(u / pf.m_tiles) * pf.expert_bytes +
-                          (int64_t)(u % pf.m_tiles) * pf.tile_bytes;
-      prefetch_l2_bulk(pf.w_gate + off, (uint32_t)pf.tile_bytes);
-      prefetch_l2_bulk(pf.w_up + off, (uint32_t)pf.tile_bytes);
+__device__ __forceinline__ bool wait_chunk(uint32_t bar, volatile int* abort_flag,
+                                           int32_t* err) {
+  if (ptx::mbar_try_wait(bar, 0)) return true;
+  const uint64_t t0 = ptx::global_timer_ns();
+  while (true) {
+    for (int i = 0; i < 64; ++i)
+      if (ptx::mbar_try_wait(bar, 0)) return true;
+    if (*abort_flag) return false;
+    if (ptx::global_timer_ns() - t0 > kSmallWaitNs) {
+      *abort_flag = 1;
+      atomicCAS(err, 0, kErrWaitTimeout);
+      return false;
     }
   }
+}
+
+// 4 consecutive x values of one token from shared memory, as fp32
+template <typename XT>
+__device__ __forceinline__ float4 ld_x4(const XT* p);
+template <>
+__device__ __forceinline__ float4 ld_x4<__nv_bfloat16>(const __nv_bfloat16* p) {
+  const uint2 v = *reinterpret_cast<const uint2*>(p);
+  return make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u),
+                     __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xffff0000u));
+}
+template <>
+__device__ __forceinline__ float4 ld_x4<float>(const float* p) {
+  return *reinterpret_cast<const float4*>(p);
+}
+
+template <typename XT, int PL>
+__global__ void __launch_bounds__(256, 1)
+    router_small_kernel(const __grid_constant__ CUtensorMap tm_w,
+                        const __grid_constant__ CUtensorMap tm_x,
+                        const float* __restrict__ bias, float* __restrict__ part,
+                        int32_t* __restrict__ counter, int32_t* __restrict__ err,
+                        float* __restrict__ logits_out, int32_t* __restrict__ idx_out,
+                        float* __restrict__ gate_out, uint8_t* __restrict__ flags, int T,
+                        int d, int E, int k, int ksplit) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + kSmallHeader - 8);
+  int* s_last = reinterpret_cast<int*>(smem + kSmallHeader - 4);
+  // chunk c: router rows [DE][256] fp32, then x rows [DG][256]
+  constexpr int kWBytes = DE * kSmallChunk * 4;
+  constexpr int kChunkBytes = kWBytes + DG * kSmallChunk * (int)sizeof(XT);
+  uint8_t* chunks = smem + kSmallHeader;
   const int g = blockIdx.x, et = blockIdx.y, z = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t t0 = (int64_t)g * DG;
-  const int64_t kbeg = (int64_t)z * ksplit;
-  const int64_t klen = min(d, kbeg + ksplit) - kbeg;
-  const int64_t v8 = klen / 8;
-  for (int64_t i = threadIdx.x; i < DG * v8; i += blockDim.x) {
-    const int tt = (int)(i / v8);
-    const int64_t kk = (i - tt * v8) * 8;
-    float* dst = xs + tt * ksplit + kk;
-    if (t0 + tt < T) {
-      load_x8<XT>(x, (t0 + tt) * d + kbeg + kk, dst);
-    } else {
-#pragma unroll
-      for (int q = 0; q < 8; ++q) dst[q] = 0.f;
-    }
+  const int t0 = g * DG, e0 = et * DE;
+  const int kbeg = z * ksplit;
+  const int klen = min(d, kbeg + ksplit) - kbeg;  // > 0, a multiple of 8
+  const int nch = (klen + kSmallChunk - 1) / kSmallChunk;
+  const int nt = min(DG, T - t0);
+  if (threadIdx.x == 0) {
+    ptx::prefetch_tensormap(&tm_w);
+    ptx::prefetch_tensormap(&tm_x);
+    for (int c = 0; c < nch; ++c) ptx::mbar_init(ptx::smem_addr(&bars[c]), 1);
+    *s_abort = 0;
+    ptx::fence_mbar_init();
   }
   __syncthreads();
-  // the 4 experts of this warp: all their router-row loads first
-  float4 wv[4][ITER];
+  griddep_wait();
+  griddep_launch_dependents();
+  if (threadIdx.x == 0) {
+    // both are re-read by other CTAs: router rows by every token group, x by
+    // every expert tile
+    const uint64_t pol = ptx::policy_evict_last();
+    for (int c = 0; c < nch; ++c) {
+      const uint32_t bar = ptx::smem_addr(&bars[c]);
+      const uint32_t dst = ptx::smem_addr(chunks + (size_t)c * kChunkBytes);
+      ptx::mbar_arrive_expect_tx(bar, (uint32_t)kChunkBytes);
+      ptx::tma_load_2d(&tm_w, dst, bar, kbeg + c * kSmallChunk, e0, pol);
+      ptx::tma_load_2d(&tm_x, dst + kWBytes, bar, kbeg + c * kSmallChunk, t0, pol);
+    }
+  }
+  float bv[PL];
+  load_bias<PL>(bias, E, lane, bv);
+
+  // Each accumulator adds its products in ascending k; columns of a chunk
+  // past this split's end are loaded but not used.
+  float acc[4][DG];
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const int e = et * DE + warp * 4 + j;
-    const float* wr = w_r + (int64_t)e * d + kbeg;
+  for (int j = 0; j < 4; ++j)
 #pragma unroll
-    for (int it = 0; it < ITER; ++it) {
-      const int64_t kk = 4 * lane + 128 * it;
-      wv[j][it] = (e < E && kk < klen) ? *reinterpret_cast<const float4*>(wr + kk)
-                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int tt = 0; tt < DG; ++tt) acc[j][tt] = 0.f;
+  for (int c = 0; c < nch; ++c) {
+    if (!wait_chunk(ptx::smem_addr(&bars[c]), s_abort, err)) break;
+    const float* wrow = reinterpret_cast<const float*>(chunks + (size_t)c * kChunkBytes) +
+                        warp * 4 * kSmallChunk;
+    const XT* xrow = reinterpret_cast<const XT*>(chunks + (size_t)c * kChunkBytes + kWBytes);
+    const int cl = min(kSmallChunk, klen - c * kSmallChunk);
+#pragma unroll
+    for (int h = 0; h < kSmallChunk / 128; ++h) {
+      if (128 * h + 4 * lane < cl) {
+        const int kk = 128 * h + 4 * lane;
+        float4 w4[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          w4[j] = *reinterpret_cast<const float4*>(wrow + j * kSmallChunk + kk);
+#pragma unroll
+        for (int tt = 0; tt < DG; ++tt) {
+          const float4 xv = ld_x4<XT>(xrow + tt * kSmallChunk + kk);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            acc[j][tt] = fmaf(w4[j].x, xv.x, acc[j][tt]);
+            acc[j][tt] = fmaf(w4[j].y, xv.y, acc[j][tt]);
+            acc[j][tt] = fmaf(w4[j].z, xv.z, acc[j][tt]);
+            acc[j][tt] = fmaf(w4[j].w, xv.w, acc[j][tt]);
+          }
+        }
+      }
     }
   }
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    const int e = et * DE + warp * 4 + j;
+    const int e = e0 + warp * 4 + j;
     if (e >= E) break;
-    float acc[DG];
-#pragma unroll
-    for (int tt = 0; tt < DG; ++tt) acc[tt] = 0.f;
-#pragma unroll
-    for (int it = 0; it < ITER; ++it) {
-      const int64_t kk = 4 * lane + 128 * it;
-      if (kk >= klen) break;
-      const float4 w4 = wv[j][it];
-#pragma unroll
-      for (int tt = 0; tt < DG; ++tt) {
-        const float4 xv = *reinterpret_cast<const float4*>(xs + tt * ksplit + kk);
-        acc[tt] = fmaf(w4.x, xv.x, acc[tt]);
-        acc[tt] = fmaf(w4.y, xv.y, acc[tt]);
-        acc[tt] = fmaf(w4.z, xv.z, acc[tt]);
-        acc[tt] = fmaf(w4.w, xv.w, acc[tt]);
-      }
-    }
 #pragma unroll
     for (int tt = 0; tt < DG; ++tt)
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1)
-        acc[tt] += __shfl_xor_sync(0xffffffffu, acc[tt], off);
-    if (lane < DG && t0 + lane < T) {
-      float v = acc[0];
+        acc[j][tt] += __shfl_xor_sync(0xffffffffu, acc[j][tt], off);
+    if (lane < nt) {
+      float v = acc[j][0];
 #pragma unroll
       for (int tt = 1; tt < DG; ++tt)
-        if (lane == tt) v = acc[tt];
+        if (lane == tt) v = acc[j][tt];
       part[((int64_t)z * T + t0 + lane) * E + e] = v;
     }
   }
   __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0)
-    s_last = atomicAdd(&counter[g], 1) == (int)(gridDim.y * gridDim.z) - 1;
+  if (threadIdx.x == 0) {
+    if (*s_abort)  // copies may still be in flight: give them the wait limit
+      for (int c = 0; c < nch; ++c) {
+        const uint64_t tw = ptx::global_timer_ns();
+        while (!ptx::mbar_try_wait(ptx::smem_addr(&bars[c]), 0))
+          if (ptx::global_timer_ns() - tw > kSmallWaitNs) break;
+      }
+    *s_last = atomicAdd(&counter[g], 1) == (int)(gridDim.y * gridDim.z) - 1;
+  }
   __syncthreads();
-  if (!s_last) return;
+  if (!*s_last) return;
   __threadfence();
-  const int64_t t = t0 + warp;
-  if (t < T) {
+  // split sums of the group's tokens into shared memory (the chunks are
+  // done): (token, expert) elements spread over the threads, each added in
+  // ascending split order; a thread has the loads of 4 elements x 8 splits in
+  // flight at once
+  float* lgs = reinterpret_cast<float*>(chunks);  // [DG][E]
+  const int nz = (int)gridDim.z;
+  const int nel = nt * E;
+  const int64_t zstride = (int64_t)T * E;
+  const float* pbase = part + (int64_t)t0 * E;  // rows t0.. are contiguous
+  for (int el0 = threadIdx.x; el0 < nel; el0 += 4 * blockDim.x) {
+    float sum[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int z0 = 0; z0 < nz; z0 += 8) {
+      float v[4][8];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int el = el0 + r * (int)blockDim.x;
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          v[r][q] = (el < nel && z0 + q < nz) ? __ldcg(pbase + (z0 + q) * zstride + el) : 0.f;
+      }
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          if (z0 + q < nz) sum[r] += v[r][q];
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int el = el0 + r * (int)blockDim.x;
+      if (el < nel) lgs[el] = sum[r];
+    }
+  }
+  __syncthreads();
+  if (warp < nt) {
     float lg[PL];
 #pragma unroll
-    for (int i = 0; i < PL; ++i) lg[i] = 0.f;
-    for (int zz = 0; zz < (int)gridDim.z; ++zz) {
-      const float* pz = part + ((int64_t)zz * T + t) * E + lane;
-#pragma unroll
-      for (int i = 0; i < PL; ++i)
-        if (lane + 32 * i < E) lg[i] += __ldcg(pz + 32 * i);
-    }
-    warp_select_token<PL>(lg, bias, logits_out, idx_out, gate_out, flags, t, E, k, lane);
+    for (int i = 0; i < PL; ++i) lg[i] = (lane + 32 * i < E) ? lgs[warp * E + lane + 32 * i] : 0.f;
+    warp_select_token<PL>(lg, bv, logits_out, idx_out, gate_out, flags, t0 + warp, E, k, lane);
   }
   if (threadIdx.x == 0) counter[g] = 0;
 }
@@ -564,12 +646,35 @@ bool router_uses_tensor_cores(const Shape& sh) {
 }
 
 constexpr int64_t kSmallRouterMaxTokens = 256;
-constexpr int64_t kPrefetchBytes = 96ll << 20;  // L2 prefetch budget of a decode call
 
 bool router_uses_small_kernel(const Shape& sh) { return sh.T <= kSmallRouterMaxTokens; }
 
-// Contraction splits of the small-batch router (<= 1024 elements each).
-int router_small_splits(const Shape& sh) { return (int)((sh.d + 1023) / 1024); }
+// Contraction split of the small-batch router: as many splits as fill the
+// SMs once with the (token group, expert tile) pairs, at least enough that a
+// CTA's rows fit its shared-memory budget, and at most one per 256 elements.
+// Returns the number of splits; *ksplit (if given) gets their length.
+int small_chunk_bytes(const Shape& sh) {
+  return DE * kSmallChunk * 4 + DG * kSmallChunk * (sh.bf16 ? 2 : 4);
+}
+
+int router_small_plan(const Shape& sh, int* ksplit_out) {
+  const int64_t base = ((sh.T + DG - 1) / DG) * ((sh.E + DE - 1) / DE);
+  int64_t chunks = (kSmallMaxBytes - kSmallHeader) / small_chunk_bytes(sh);
+  if (chunks > kSmallMaxChunks) chunks = kSmallMaxChunks;
+  const int64_t kmax = chunks * kSmallChunk;
+  int64_t n = num_sms() / base;
+  const int64_t n_min = (sh.d + kmax - 1) / kmax;
+  const int64_t n_max = (sh.d + kSmallChunk - 1) / kSmallChunk;
+  if (n > n_max) n = n_max;
+  if (n < n_min) n = n_min;
+  if (n < 1) n = 1;
+  int64_t ks = (sh.d + n - 1) / n;
+  ks = (ks + 31) / 32 * 32;
+  if (ksplit_out) *ksplit_out = (int)ks;
+  return (int)((sh.d + ks - 1) / ks);
+}
+
+int router_small_splits(const Shape& sh) { return router_small_plan(sh, nullptr); }
 
 int router_launch_count(const Shape& sh) {
   return router_uses_tensor_cores(sh) ? 3 : (router_uses_small_kernel(sh) ? 1 : 2);
@@ -586,11 +691,69 @@ int router_splits(const Shape& sh) {
   return (int)want;
 }
 
+PFN_cuTensorMapEncodeTiled_v12000 router_map_encoder() {
+  static std::atomic<PFN_cuTensorMapEncodeTiled_v12000> fn{nullptr};
+  if (!fn.load()) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn.store(reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p));
+  }
+  return fn.load();
+}
+
+// Tensor maps of the small-batch router: router rows [E, d] fp32 in boxes of
+// 32 rows x 256 columns, x [T, d] in boxes of 8 rows x 256 columns; no
+// swizzle, out-of-range elements read as zero.
+bool make_router_maps(const Shape& sh, const void* x, const float* w_r, CUtensorMap* tm_w,
+                      CUtensorMap* tm_x) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = router_map_encoder();
+  if (!enc) return false;
+  const cuuint32_t estr[2] = {1, 1};
+  const cuuint64_t wdims[2] = {(cuuint64_t)sh.d, (cuuint64_t)sh.E};
+  const cuuint64_t wstr[1] = {(cuuint64_t)sh.d * 4};
+  const cuuint32_t wbox[2] = {(cuuint32_t)kSmallChunk, (cuuint32_t)DE};
+  if (enc(tm_w, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(w_r), wdims, wstr, wbox,
+          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  const int es = sh.bf16 ? 2 : 4;
+  const cuuint64_t xdims[2] = {(cuuint64_t)sh.d, (cuuint64_t)sh.T};
+  const cuuint64_t xstr[1] = {(cuuint64_t)sh.d * es};
+  const cuuint32_t xbox[2] = {(cuuint32_t)kSmallChunk, (cuuint32_t)DG};
+  return enc(tm_x, sh.bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+             2, const_cast<void*>(x), xdims, xstr, xbox, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename XT, int PL>
+cudaError_t launch_small(dim3 grid, size_t smem, cudaStream_t st, const CUtensorMap& tm_w,
+                         const CUtensorMap& tm_x, const float* bias, float* part, int32_t* counter, int32_t* err,
+                         float* logits_out, int32_t* idx, float* gate, uint8_t* flags, int T,
+                         int d, int E, int k, int ksplit) {
+  // the shared-memory limit is raised once per device and instantiation
+  static std::atomic<uint64_t> attr_set{0};
+  int dev = 0;
+  cudaError_t a = cudaGetDevice(&dev);
+  if (a != cudaSuccess) return a;
+  const uint64_t bit = 1ull << (dev & 63);
+  if (!(attr_set.load() & bit)) {
+    a = cudaFuncSetAttribute(router_small_kernel<XT, PL>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, kSmallMaxBytes);
+    if (a != cudaSuccess) return a;
+    attr_set.fetch_or(bit);
+  }
+  return launch_pdl(router_small_kernel<XT, PL>, grid, dim3(256), smem, st, tm_w, tm_x, bias,
+                    part, counter, err, logits_out, idx, gate, flags, T, d, E, k, ksplit);
+}
+
 cudaError_t launch_router(const Shape& sh, const void* x, const float* w_r,
                           const float* bias, float* part, int32_t* idx,
                           float* gate, uint8_t* flags, float* logits_out,
                           void* planes, int32_t* plan, int32_t* err,
-                          const void* prefetch_gate, const void* prefetch_up,
                           cudaStream_t st) {
   int n_outer, n_inner;
   int64_t outer_stride, inner_stride, row_stride;
@@ -598,38 +761,20 @@ cudaError_t launch_router(const Shape& sh, const void* x, const float* w_r,
   if (router_uses_small_kernel(sh)) {
     // one launch: logits, split sums and top-k; the group counters live in
     // the workspace header after the error word (zero between calls)
-    const int nsplit = router_small_splits(sh);
-    const int64_t steps = ((sh.d + nsplit - 1) / nsplit + 127) / 128;  // <= 8
-    const int iter = steps <= 1 ? 1 : steps <= 2 ? 2 : steps <= 4 ? 4 : 8;
-    const int64_t ksplit = 128 * (int64_t)iter;
+    int ksplit = 0;
+    const int nsplit = router_small_plan(sh, &ksplit);
     const dim3 grid((unsigned)((sh.T + DG - 1) / DG), (unsigned)((sh.E + DE - 1) / DE),
                     (unsigned)nsplit);
-    const size_t smem = (size_t)DG * ksplit * sizeof(float);
+    const size_t smem = (size_t)kSmallHeader +
+                        (size_t)((ksplit + kSmallChunk - 1) / kSmallChunk) * small_chunk_bytes(sh);
+    CUtensorMap tm_w, tm_x;
+    if (!make_router_maps(sh, x, w_r, &tm_w, &tm_x)) return cudaErrorInvalidValue;
     int32_t* counter = err + 2;
-    WeightPrefetch pf;
-    const bool aligned = ((reinterpret_cast<uintptr_t>(prefetch_gate) |
-                           reinterpret_cast<uintptr_t>(prefetch_up)) & 15) == 0;
-    if (prefetch_gate && prefetch_up && aligned && sh.T <= 64 && sh.N > 0 &&
-        expert_ffn_uses_tensor_cores(sh)) {
-      pf.w_gate = static_cast<const uint8_t*>(prefetch_gate);
-      pf.w_up = static_cast<const uint8_t*>(prefetch_up);
-      pf.expert_bytes = sh.F * sh.d * 2;
-      pf.tile_bytes = 128 * sh.d * 2;
-      pf.m_tiles = (int)(sh.F / 128);
-      const int64_t budget = kPrefetchBytes / (2 * pf.tile_bytes);  // tiles per matrix
-      const int64_t all = sh.N * pf.m_tiles;
-      pf.units = (int)(budget < all ? budget : all);
-    }
     const int pl = (int)((sh.E + 31) / 32);
     const int E = (int)sh.E, k = (int)sh.k;
-#define MOE_SMALL_IT(XT, P, I)                                                        \
-  launch_pdl(router_small_kernel<XT, P, I>, grid, dim3(256), smem, st,                \
-             static_cast<const XT*>(x), w_r, bias, part, counter, logits_out, idx, gate, \
-             flags, sh.T, sh.d, E, k, ksplit, pf)
-#define MOE_SMALL(XT, P)                                          \
-  (iter == 1 ? MOE_SMALL_IT(XT, P, 1)                             \
-   : iter == 2 ? MOE_SMALL_IT(XT, P, 2)                           \
-   : iter == 4 ? MOE_SMALL_IT(XT, P, 4) : MOE_SMALL_IT(XT, P, 8))
+#define MOE_SMALL(XT, P)                                                                \
+  launch_small<XT, P>(grid, smem, st, tm_w, tm_x, bias, part, counter, err, logits_out, idx, \
+                      gate, flags, (int)sh.T, (int)sh.d, E, k, ksplit)
 #define MOE_SMALL_PL(XT)                    \
   (pl <= 1    ? MOE_SMALL(XT, 1)            \
    : pl <= 2  ? MOE_SMALL(XT, 2)            \
@@ -640,7 +785,6 @@ cudaError_t launch_router(const Shape& sh, const void* x, const float* w_r,
     e = sh.bf16 ? MOE_SMALL_PL(__nv_bfloat16) : MOE_SMALL_PL(float);
 #undef MOE_SMALL_PL
 #undef MOE_SMALL
-#undef MOE_SMALL_IT
     return e;
   }
   if (router_uses_tensor_cores(sh)) {

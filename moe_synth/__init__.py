@@ -85,6 +85,10 @@ CONFIGS: Dict[str, MoEShape] = {
                                n_zero=8, top_k=8, ffn=1024),
     "profile_prefill": MoEShape("profile_prefill", T=4096, d=4096, n_routed=32,
                                 n_zero=8, top_k=8, ffn=1024, routing="zipf"),
+    # the decode layer's router (T=64, 160 experts) with narrow experts, so
+    # that a profiler capture holds ~0.4 GB of weights
+    "profile_router": MoEShape("profile_router", T=64, d=4096, n_routed=128,
+                               n_zero=32, top_k=8, ffn=128),
     # the large-expert layer's density (~270 rows per expert), 32 experts
     "profile_large_e": MoEShape("profile_large_e", T=1024, d=6144, n_routed=32,
                                 n_zero=8, top_k=12, ffn=2048),
