@@ -238,21 +238,18 @@ def event_time_ms(fn, reps, stream):
 
 def run_gpu(args, sh):
     import expert_routing_dispatch_router_b200 as moe
-    import torch.distributed as dist
+    from expert_routing_dispatch_router_b200 import replicas
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    pre = replicas.rank_info()
+    local = pre.local
     torch.cuda.set_device(local)
-    if world > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+    info = replicas.init("nccl", 120.0, torch.device("cuda", local))
+    world, rank = info.world, info.rank
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream()
     pk = peaks()
 
-    inp = make_inputs(sh, args.seed + rank)
+    inp = make_inputs(sh, replicas.batch_seed(args.seed, info))
     d = inp.to(dev)
     ls = moe.LayerShape(sh.T, sh.d, sh.n_routed, sh.n_zero, sh.top_k, sh.ffn,
                         torch_dtype(sh.act_dtype), sh.routed_scale)
@@ -299,8 +296,7 @@ def run_gpu(args, sh):
             step()
     graph.replay()
     torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
+    replicas.barrier(info)
     torch.cuda.synchronize()
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
@@ -310,17 +306,12 @@ def run_gpu(args, sh):
     end.record(stream)
     torch.cuda.synchronize()
     del graph
-    if world > 1:
-        dist.barrier()
+    replicas.barrier(info)
     torch.cuda.synchronize()
     clocks = sampler.stop()
-    ms = start.elapsed_time(end)
-    if world > 1:
-        tt = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = replicas.max_over_ranks(start.elapsed_time(end), info, dev)
     ms_per_step = ms / args.steps
-    value = world * args.steps * sh.T / (ms / 1e3)
+    value = replicas.job_throughput(sh.T, args.steps, info, ms)
 
     # ---- end to end through the host-buffer entry point
     x_host = inp.x.clone().pin_memory()
@@ -333,13 +324,8 @@ def run_gpu(args, sh):
     for _ in range(max(args.warmup, 3)):
         step_host()
     torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    e2e_ms = event_time_ms(step_host, args.steps, stream)
-    if world > 1:
-        tt = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+    replicas.barrier(info)
+    e2e_ms = replicas.max_over_ranks(event_time_ms(step_host, args.steps, stream), info, dev)
     assert torch.equal(out_host, out.cpu()), "host entry point disagrees with device entry point"
     act_b = sh.T * sh.d * d.x.element_size()
 
@@ -409,7 +395,7 @@ def run_gpu(args, sh):
                              "stream from HBM every step",
                        "parallelism": f"replicas{world}",
                        "launch": f"CUDA graph of {G} layer calls, replayed {args.steps // G} times"},
-            "e2e": {"value": world * sh.T / (e2e_ms / 1e3), "unit": "tokens/s",
+            "e2e": {"value": replicas.job_throughput(sh.T, 1, info, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": act_b, "d2h_bytes_per_step": act_b},
             "gpu_launches": args.steps * moe.launch_count(ls),
             "roofline": roof,
@@ -419,9 +405,7 @@ def run_gpu(args, sh):
         if not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(sh, inp)
         print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    replicas.finalize(info)
 
 
 def main():
