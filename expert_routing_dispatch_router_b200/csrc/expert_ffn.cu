@@ -201,7 +201,49 @@ __device__ __forceinline__ void wait_cleanup(uint32_t bar, uint32_t parity) {
     if (ptx::global_timer_ns() - t0 > kWaitLimitNs) return;
 }
 
-__device__ __forceinline__ float silu_f(float z) { return z / (1.0f + __expf(-z)); }
+// silu(z) = z / (1 + e^-z); the fast divide's 2-ulp error is far below the
+// bf16 rounding of h that follows (and it returns 0 once 1 + e^-z overflows,
+// where silu is 0 to fp32 precision anyway)
+__device__ __forceinline__ float silu_f(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
+
+// SwiGLU epilogue of one epilogue warp's share of a gate/up accumulator: its
+// 32-column chunks c0 = 32 eh + 64 q (q < NQ, c0 < n_cols) are read from TMEM
+// (gate at column c0, up at bn_off + c0) and become bf16 h in registers. Then
+// release() hands the accumulator back to the MMA warp, and only after that
+// are the rows stored: the next unit's MMAs do not wait for the stores.
+template <int NQ, typename Release>
+__device__ __forceinline__ void swiglu_epilogue(uint32_t tb, uint32_t bn_off, int eh,
+                                                int n_cols, int n_valid, __nv_bfloat16* outp,
+                                                int64_t out_cols, Release release) {
+  uint32_t hb[NQ][16];
+#pragma unroll
+  for (int q = 0; q < NQ; ++q) {
+    const int c0 = 32 * eh + 64 * q;
+    if (c0 < n_cols) {  // warp-uniform
+      float g[32], v[32];
+      ptx::tmem_ld32x2(tb + c0, tb + bn_off + c0, g, v);
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const __nv_bfloat162 p = __floats2bfloat162_rn(silu_f(g[2 * c]) * v[2 * c],
+                                                       silu_f(g[2 * c + 1]) * v[2 * c + 1]);
+        hb[q][c] = *reinterpret_cast<const uint32_t*>(&p);
+      }
+    }
+  }
+  release();
+  uint16_t* o16 = reinterpret_cast<uint16_t*>(outp);
+#pragma unroll
+  for (int q = 0; q < NQ; ++q) {
+    const int c0 = 32 * eh + 64 * q;
+    if (c0 < n_cols) {
+#pragma unroll
+      for (int c = 0; c < 32; ++c)
+        if (c0 + c < n_valid)
+          o16[(int64_t)(c0 + c) * out_cols] =
+              (c & 1) ? (uint16_t)(hb[q][c >> 1] >> 16) : (uint16_t)(hb[q][c >> 1] & 0xffffu);
+    }
+  }
+}
 
 template <bool GATEUP, int BN_>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -386,27 +428,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t col = (int64_t)un.m * BM + lrow;
       const int64_t obase = (int64_t)un.row0 * args.out_cols + col;
       // 32-column chunks, alternating between the two warps of this quarter
-      for (int c0 = 32 * eh; c0 < un.n_mma; c0 += 64) {
-        float g[32], v[32];
-        if (GATEUP) {
-          ptx::tmem_ld32x2(tb + c0, tb + BN + c0, g, v);
-          __nv_bfloat16* outp = static_cast<__nv_bfloat16*>(args.out) + obase;
-#pragma unroll
-          for (int c = 0; c < 32; ++c)
-            if (c0 + c < un.n_valid)
-              outp[(int64_t)(c0 + c) * args.out_cols] =
-                  __float2bfloat16_rn(silu_f(g[c]) * v[c]);
-        } else {
+      auto release = [&]() {
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(tempty_bar(acc));
+      };
+      if (GATEUP) {
+        swiglu_epilogue<BN / 64>(tb, BN, eh, un.n_mma, un.n_valid,
+                                 static_cast<__nv_bfloat16*>(args.out) + obase, args.out_cols,
+                                 release);
+      } else {
+        for (int c0 = 32 * eh; c0 < un.n_mma; c0 += 64) {
+          float g[32];
           ptx::tmem_ld32(tb + c0, g);
           float* outp = static_cast<float*>(args.out) + obase;
 #pragma unroll
           for (int c = 0; c < 32; ++c)
             if (c0 + c < un.n_valid) outp[(int64_t)(c0 + c) * args.out_cols] = g[c];
         }
+        release();
       }
-      ptx::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(tempty_bar(acc));
       if (++acc == C::kAccBufs) {
         acc = 0;
         acc_phase ^= 1u;
@@ -647,31 +688,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                           (uint32_t)acc * kAccStride;
       const int64_t col = (int64_t)un.m * 2 * BM + (int64_t)rank * BM + lrow;
       const int64_t obase = (int64_t)un.row0 * args.out_cols + col;
-      for (int c0 = 32 * eh; c0 < n_pair; c0 += 64) {
-        float g[32], v[32];
-        if (GATEUP) {
-          ptx::tmem_ld32x2(tb + c0, tb + BN + c0, g, v);
-          __nv_bfloat16* outp = static_cast<__nv_bfloat16*>(args.out) + obase;
-#pragma unroll
-          for (int c = 0; c < 32; ++c)
-            if (c0 + c < un.n_valid)
-              outp[(int64_t)(c0 + c) * args.out_cols] =
-                  __float2bfloat16_rn(silu_f(g[c]) * v[c]);
-        } else {
+      auto release = [&]() {
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (leader)
+            ptx::mbar_arrive(tempty_bar(acc));
+          else
+            ptx::mbar_arrive_remote(ptx::map_to_rank(tempty_bar(acc), 0));
+        }
+      };
+      if (GATEUP) {
+        swiglu_epilogue<BN / 64>(tb, BN, eh, n_pair, un.n_valid,
+                                 static_cast<__nv_bfloat16*>(args.out) + obase, args.out_cols,
+                                 release);
+      } else {
+        for (int c0 = 32 * eh; c0 < n_pair; c0 += 64) {
+          float g[32];
           ptx::tmem_ld32(tb + c0, g);
           float* outp = static_cast<float*>(args.out) + obase;
 #pragma unroll
           for (int c = 0; c < 32; ++c)
             if (c0 + c < un.n_valid) outp[(int64_t)(c0 + c) * args.out_cols] = g[c];
         }
-      }
-      ptx::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        if (leader)
-          ptx::mbar_arrive(tempty_bar(acc));
-        else
-          ptx::mbar_arrive_remote(ptx::map_to_rank(tempty_bar(acc), 0));
+        release();
       }
       if (++acc == C::kAccBufs) {
         acc = 0;
