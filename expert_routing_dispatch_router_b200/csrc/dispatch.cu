@@ -185,7 +185,8 @@ __global__ void __launch_bounds__(1024)
                           int W, int32_t* __restrict__ counts,
                           int32_t* __restrict__ offsets, int32_t* __restrict__ row_token,
                           int32_t* __restrict__ slot_row, int64_t rows_cap,
-                          int32_t* err) {
+                          int32_t* err, int32_t* __restrict__ tile_start, int tile_gu,
+                          int tile_dn) {
   extern __shared__ uint32_t sm[];
   uint32_t* mask = sm;
   int32_t* pre = reinterpret_cast<int32_t*>(sm + (size_t)E * W);
@@ -228,6 +229,19 @@ __global__ void __launch_bounds__(1024)
   }
   if (threadIdx.x == 0) offsets[N] = R;
   __syncthreads();
+  if (tile_start) {
+    // the expert GEMMs' plans: token-tile prefixes of both GEMMs (v is the
+    // count of routed expert threadIdx.x, 0 past N)
+    int32_t tot = 0;
+    const int32_t g = block_exclusive_scan((v + tile_gu - 1) / tile_gu, warp_sums, &tot);
+    if ((int)threadIdx.x < N) tile_start[threadIdx.x] = g;
+    if (threadIdx.x == 0) tile_start[N] = tot;
+    __syncthreads();
+    const int32_t dn = block_exclusive_scan((v + tile_dn - 1) / tile_dn, warp_sums, &tot);
+    if ((int)threadIdx.x < N) tile_start[N + 1 + threadIdx.x] = dn;
+    if (threadIdx.x == 0) tile_start[2 * N + 1] = tot;
+    __syncthreads();
+  }
   for (int t = threadIdx.x; t < T; t += blockDim.x) {
     const int w = t >> 5;
     const uint32_t below = (1u << (t & 31)) - 1u;
@@ -278,6 +292,8 @@ bool dispatch_small_fits(const Shape& sh) {
   return sh.T <= 4096 && dispatch_small_smem(sh) <= kSmallDispatchSmem;
 }
 
+bool dispatch_plans_tiles(const Shape& sh) { return dispatch_small_fits(sh); }
+
 int dispatch_launch_count(const Shape& sh) {
   return (dispatch_small_fits(sh) ? 1 : 3) + (sh.N > 0 ? 1 : 0);
 }
@@ -297,7 +313,8 @@ cudaError_t launch_dispatch(const Shape& sh, const void* x, const int32_t* idx,
                             int32_t* chunk_base, int32_t* counts,
                             int32_t* offsets, int32_t* row_token,
                             int32_t* slot_row, void* x_perm, int32_t* err,
-                            cudaStream_t st) {
+                            cudaStream_t st, int32_t* tile_start, int tile_gu,
+                            int tile_dn) {
   const int E = (int)sh.E, N = (int)sh.N, k = (int)sh.k;
   cudaError_t e = cudaSuccess;
   if (dispatch_small_fits(sh)) {
@@ -312,7 +329,8 @@ cudaError_t launch_dispatch(const Shape& sh, const void* x, const int32_t* idx,
       attr_set = true;
     }
     e = launch_pdl(dispatch_small_kernel, dim3(1), dim3(1024), smem, st, idx, (int)sh.T,
-                   k, E, N, W, counts, offsets, row_token, slot_row, sh.T * sh.k, err);
+                   k, E, N, W, counts, offsets, row_token, slot_row, sh.T * sh.k, err,
+                   tile_start, tile_gu, tile_dn);
     if (e != cudaSuccess) return e;
   } else {
     const size_t smem = (size_t)E * kWords * sizeof(uint32_t);
@@ -327,7 +345,7 @@ cudaError_t launch_dispatch(const Shape& sh, const void* x, const int32_t* idx,
                    sh.T, k, E, N, chunk_base, offsets, row_token, slot_row);
     if (e != cudaSuccess) return e;
   }
-  if (N > 0) {
+  if (N > 0 && x_perm) {  // no x_perm: the GEMM gathers the rows itself
     const int64_t vpr = sh.d * sh.es / 16;
     int64_t rows = sh.T * sh.k;
     int64_t blocks = (rows + 7) / 8;

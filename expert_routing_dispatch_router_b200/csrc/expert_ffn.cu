@@ -142,6 +142,12 @@ struct GemmArgs {
   int a_rows;    // rows of A per expert (A row = e * a_rows + (m % mt_chunk) * BM)
   int mt_chunk;  // m-tiles per contraction chunk: m-tile m covers k-blocks
   int kb_chunk;  // [(m / mt_chunk) * kb_chunk, +kb_chunk) with a fresh accumulator
+  // Gate/up of the fused layer (single-CTA path): when set, token rows are
+  // gathered from x by row_token with TMA gather4 (tmB16 is then x's map with
+  // a one-row box) instead of being read from x_perm; oob_row is a row outside
+  // x, which reads as zeros, for the padding rows of a tile.
+  const int32_t* row_token = nullptr;
+  int oob_row = 0;
 };
 
 struct Unit {
@@ -269,6 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* s_tiles = reinterpret_cast<int*>(smem + C::kTabOff);
   int* s_offs = s_tiles + (kMaxExperts + 1);
+  __shared__ int s_ids[BN_];  // token ids of the current unit's rows (gather)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int N = args.N;
@@ -311,20 +318,43 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ---------------------------------------------------- TMA producer --
-    if (lane == 0) {
-      // L2 policy per unit: an expert with a single token tile reads each
-      // weight tile once (a decode step), so its weights are streamed
-      // evict-first and its few token rows kept evict-last. An expert with
-      // several token tiles reuses every weight tile once per token tile, so
-      // both operands use the normal policy.
-      const uint64_t pol_first = ptx::policy_evict_first();
-      const uint64_t pol_last = ptx::policy_evict_last();
-      const uint64_t pol_normal = ptx::policy_evict_normal();
-      int stage = 0;
-      uint32_t phase = 0, armed = 0, armed_par = 0;
-      bool ok = true;
-      for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
-        const Unit un = decode_unit<BN>(u, s_tiles, s_offs, N, args.m_tiles);
+    // Lane 0 issues the copies. When the token rows are gathered from x, the
+    // whole warp fetches the token ids one unit ahead (lane + 32 i of the next
+    // unit's rows), so the copies never wait for them.
+    const bool gather = GATEUP && args.row_token != nullptr;
+    constexpr int kIds = BN / 32;
+    int nxt[kIds];
+    auto fetch_ids = [&](int u) {
+      if (u < total_units) {
+        const Unit nu = decode_unit<BN>(u, s_tiles, s_offs, N, args.m_tiles);
+#pragma unroll
+        for (int i = 0; i < kIds; ++i) {
+          const int j = lane + 32 * i;  // padding rows read a row outside x: zeros
+          nxt[i] = j < nu.n_valid ? __ldg(args.row_token + nu.row0 + j) : args.oob_row;
+        }
+      }
+    };
+    if (gather) fetch_ids(blockIdx.x);
+    // L2 policy per unit: an expert with a single token tile reads each
+    // weight tile once (a decode step), so its weights are streamed
+    // evict-first and its few token rows kept evict-last. An expert with
+    // several token tiles reuses every weight tile once per token tile, so
+    // both operands use the normal policy.
+    const uint64_t pol_first = ptx::policy_evict_first();
+    const uint64_t pol_last = ptx::policy_evict_last();
+    const uint64_t pol_normal = ptx::policy_evict_normal();
+    int stage = 0;
+    uint32_t phase = 0, armed = 0, armed_par = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
+      const Unit un = decode_unit<BN>(u, s_tiles, s_offs, N, args.m_tiles);
+      if (gather) {
+#pragma unroll
+        for (int i = 0; i < kIds; ++i) s_ids[lane + 32 * i] = nxt[i];
+        __syncwarp();
+        fetch_ids(u + (int)gridDim.x);
+      }
+      if (lane == 0) {
         const int arow = un.e * args.a_rows + (un.m % args.mt_chunk) * BM;
         const int kb0 = (un.m / args.mt_chunk) * args.kb_chunk;
         const uint32_t bytes = C::kNumA * kTileBytes + (uint32_t)un.n_mma * 128u;
@@ -340,13 +370,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t a0 = sbase + stage * C::kStageBytes;
           ptx::tma_load_2d(&tmA0, a0, fb, kb * BK, arow, pol_w);
           if (GATEUP) ptx::tma_load_2d(&tmA1, a0 + kTileBytes, fb, kb * BK, arow, pol_w);
-          // token rows: 128-row boxes while 128 or more remain, then 16-row boxes
+          // token rows: 128-row boxes while 128 or more remain, then 16-row
+          // boxes; or, gathering from x, four rows per request
           const uint32_t b0 = a0 + C::kNumA * kTileBytes;
-          int j = 0;
-          for (; j + 128 <= un.n_mma; j += 128)
-            ptx::tma_load_2d(&tmB128, b0 + j * 128u, fb, kb * BK, un.row0 + j, pol_x);
-          for (; j < un.n_mma; j += 16)
-            ptx::tma_load_2d(&tmB16, b0 + j * 128u, fb, kb * BK, un.row0 + j, pol_x);
+          if (gather) {
+            for (int j = 0; j < un.n_mma; j += 4)
+              ptx::tma_gather4_2d(&tmB16, b0 + j * 128u, fb, kb * BK, s_ids[j], s_ids[j + 1],
+                                  s_ids[j + 2], s_ids[j + 3], pol_x);
+          } else {
+            int j = 0;
+            for (; j + 128 <= un.n_mma; j += 128)
+              ptx::tma_load_2d(&tmB128, b0 + j * 128u, fb, kb * BK, un.row0 + j, pol_x);
+            for (; j < un.n_mma; j += 16)
+              ptx::tma_load_2d(&tmB16, b0 + j * 128u, fb, kb * BK, un.row0 + j, pol_x);
+          }
           armed |= 1u << stage;
           armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
           if (++stage == S) {
@@ -355,10 +392,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (!ok) {  // let our own loads land before the CTA goes away
-        for (int s = 0; s < S; ++s)
-          if ((armed >> s) & 1u) wait_cleanup(full_bar(s), (armed_par >> s) & 1u);
-      }
+      // every lane follows lane 0 (and keeps s_ids until its copies are issued)
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+    }
+    if (lane == 0 && !ok) {  // let our own loads land before the CTA goes away
+      for (int s = 0; s < S; ++s)
+        if ((armed >> s) & 1u) wait_cleanup(full_bar(s), (armed_par >> s) & 1u);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------ MMA issuer --
@@ -966,11 +1005,22 @@ int expert_ffn_launch_count(const Shape& sh) {
   return expert_ffn_uses_tensor_cores(sh) ? 3 : 2;
 }
 
+void expert_ffn_tiles(const Shape& sh, int* tile_gu, int* tile_dn) {
+  const bool pairs = use_pairs(sh);
+  *tile_gu = pairs ? 256 : tile_gateup_for(sh.T);
+  *tile_dn = pairs ? 256 : tile_down_for(sh.T);
+}
+
+bool expert_ffn_gathers(const Shape& sh) {
+  return expert_ffn_uses_tensor_cores(sh) && !use_pairs(sh) && tile_gateup_for(sh.T) <= 128;
+}
+
 cudaError_t launch_expert_ffn(const Shape& sh, const void* x_perm,
                               const int32_t* offsets, const void* w_gate,
                               const void* w_up, const void* w_down, void* h,
                               void* y_perm, int32_t* tile_start, int32_t* err,
-                              cudaStream_t st) {
+                              cudaStream_t st, const void* x_src,
+                              const int32_t* row_token, bool plan_ready) {
   if (sh.N == 0 || sh.T == 0) return cudaSuccess;
   if (!expert_ffn_uses_tensor_cores(sh)) {
     if (sh.bf16)
@@ -991,11 +1041,14 @@ cudaError_t launch_expert_ffn(const Shape& sh, const void* x_perm,
   if (!ok) return cudaErrorInvalidValue;
 
   const bool pairs = use_pairs(sh);
-  const int tgu = pairs ? 256 : tile_gateup_for(sh.T);
-  const int tdn = pairs ? 256 : tile_down_for(sh.T);
-  cudaError_t e = launch_pdl(gemm_plan_kernel, dim3(1), dim3(1024), 0, st, offsets,
-                             (int)sh.N, tgu, tdn, tile_start);
-  if (e != cudaSuccess) return e;
+  int tgu = 0, tdn = 0;
+  expert_ffn_tiles(sh, &tgu, &tdn);
+  cudaError_t e = cudaSuccess;
+  if (!plan_ready) {
+    e = launch_pdl(gemm_plan_kernel, dim3(1), dim3(1024), 0, st, offsets, (int)sh.N, tgu, tdn,
+                   tile_start);
+    if (e != cudaSuccess) return e;
+  }
 
   GemmArgs gu;
   gu.offsets = offsets;
@@ -1009,6 +1062,13 @@ cudaError_t launch_expert_ffn(const Shape& sh, const void* x_perm,
   gu.a_rows = gu.out_cols;
   gu.mt_chunk = gu.m_tiles;
   gu.kb_chunk = gu.num_kb;
+  if (x_src && row_token) {
+    // token rows straight from x: x16 becomes x's one-row-box map
+    if (!expert_ffn_gathers(sh) || !make_map(&x16, x_src, (uint64_t)sh.T, (uint64_t)sh.d, 1))
+      return cudaErrorInvalidValue;
+    gu.row_token = row_token;
+    gu.oob_row = (int)sh.T;
+  }
   if (pairs) {
     GemmArgs gp = gu;
     gp.m_tiles = (int)(sh.F / 256);  // pairs of 128-row tiles

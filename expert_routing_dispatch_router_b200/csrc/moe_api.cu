@@ -119,12 +119,22 @@ moe_status_t run_layer(const Shape& sh, const void* x, const float* w_router,
                                 gate, nullptr, nullptr, at<void>(ws, L.planes),
                                 at<int32_t>(ws, L.router_plan), err, st);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
+  // where the gate/up GEMM gathers token rows itself, x_perm is never written
+  const bool gather = expert_ffn_gathers(sh);
+  // the one-block dispatch also writes the expert GEMMs' plans
+  const bool plan = sh.N > 0 && expert_ffn_uses_tensor_cores(sh) && dispatch_plans_tiles(sh);
+  int tgu = 0, tdn = 0;
+  expert_ffn_tiles(sh, &tgu, &tdn);
+  int32_t* row_token = at<int32_t>(ws, L.row_token);
+  int32_t* tile_start = at<int32_t>(ws, L.tile_start);
   e = launch_dispatch(sh, x, idx, at<int32_t>(ws, L.chunk_base),
-                      counts ? counts : at<int32_t>(ws, L.counts), offsets,
-                      at<int32_t>(ws, L.row_token), slot_row, x_perm, err, st);
+                      counts ? counts : at<int32_t>(ws, L.counts), offsets, row_token,
+                      slot_row, gather ? nullptr : x_perm, err, st, plan ? tile_start : nullptr,
+                      tgu, tdn);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   e = launch_expert_ffn(sh, x_perm, offsets, w_gate, w_up, w_down, at<void>(ws, L.h),
-                        y_perm, at<int32_t>(ws, L.tile_start), err, st);
+                        y_perm, tile_start, err, st, gather ? x : nullptr,
+                        gather ? row_token : nullptr, plan);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   e = launch_combine(sh, x, y_perm, idx, gate, slot_row, out, st);
   return cuda_status(e);
@@ -312,7 +322,10 @@ int32_t moe_layer_launch_count(const moe_config_t* cfg) {
   if (make_shape(cfg, &sh) != MOE_OK || sh.T == 0) return 0;
   int32_t n = router_launch_count(sh);  // (split + GEMM | logits) + top-k
   n += dispatch_launch_count(sh);  // (count, scan, scatter | small) + gather
+  if (sh.N > 0 && expert_ffn_gathers(sh)) n -= 1;  // the gate/up GEMM gathers
   n += expert_ffn_launch_count(sh);
+  if (sh.N > 0 && expert_ffn_uses_tensor_cores(sh) && dispatch_plans_tiles(sh))
+    n -= 1;  // the one-block dispatch writes the GEMM plans
   n += 1;                         // combine
   return n;
 }

@@ -64,16 +64,28 @@ cudaError_t launch_router(const Shape& sh, const void* x, const float* w_r,
                           float* gate, uint8_t* flags, float* logits_out,
                           void* planes, int32_t* plan, int32_t* err,
                           cudaStream_t st);
+// x_perm null: the rows are not gathered (the gate/up GEMM gathers them).
+// tile_start given and dispatch_plans_tiles(sh): the one-block dispatch also
+// writes the expert GEMMs' token-tile prefixes for tiles tile_gu and tile_dn.
 cudaError_t launch_dispatch(const Shape& sh, const void* x, const int32_t* idx,
                             int32_t* chunk_base, int32_t* counts,
                             int32_t* offsets, int32_t* row_token,
                             int32_t* slot_row, void* x_perm, int32_t* err,
-                            cudaStream_t st);
+                            cudaStream_t st, int32_t* tile_start = nullptr,
+                            int tile_gu = 0, int tile_dn = 0);
+bool dispatch_plans_tiles(const Shape& sh);
+// With x_src and row_token given (the fused layer, where expert_ffn_gathers
+// holds), the gate/up GEMM reads token rows from x by row_token and x_perm is
+// not used.
 cudaError_t launch_expert_ffn(const Shape& sh, const void* x_perm,
                               const int32_t* offsets, const void* w_gate,
                               const void* w_up, const void* w_down, void* h,
                               void* y_perm, int32_t* tile_start, int32_t* err,
-                              cudaStream_t st);
+                              cudaStream_t st, const void* x_src = nullptr,
+                              const int32_t* row_token = nullptr, bool plan_ready = false);
+bool expert_ffn_gathers(const Shape& sh);
+// Token tiles of the gate/up and down GEMMs on the tensor-core path.
+void expert_ffn_tiles(const Shape& sh, int* tile_gu, int* tile_dn);
 cudaError_t launch_combine(const Shape& sh, const void* x, const void* y_perm,
                            const int32_t* idx, const float* gate,
                            const int32_t* slot_row, void* out, cudaStream_t st);

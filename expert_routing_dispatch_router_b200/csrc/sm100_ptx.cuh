@@ -66,6 +66,21 @@ __device__ __forceinline__ void tma_load_2d(const CUtensorMap* map, uint32_t dst
       : "memory");
 }
 
+// 2-D gather of four rows: rows y0..y3 of the tensor, columns [x, x + box
+// width), land as four consecutive box rows at `dst` (swizzled as a tiled load
+// to the same address would be). The tensor map's box is one row high. Rows
+// outside the tensor read as zero.
+__device__ __forceinline__ void tma_gather4_2d(const CUtensorMap* map, uint32_t dst,
+                                               uint32_t bar, int32_t x, int32_t y0, int32_t y1,
+                                               int32_t y2, int32_t y3, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::"
+      "bytes.L2::cache_hint [%0], [%1, {%3, %4, %5, %6, %7}], [%2], %8;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y0), "r"(y1), "r"(y2),
+      "r"(y3), "l"(policy)
+      : "memory");
+}
+
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));

@@ -55,11 +55,14 @@ def test_workspace_size_valid_and_invalid(L):
 
 def test_launch_count(L):
     # router 1 (T <= 256), 2 (CUDA cores) or 3 (split + tensor-core GEMM +
-    # top-k), dispatch 1 (one block for small T) or 3, + gather, FFN 3
-    # (tcgen05) or 2 (CUDA cores), combine 1
-    assert L.moe_layer_launch_count(ctypes.byref(cfg())) == 1 + 2 + 3 + 1
+    # top-k); dispatch 1 (one block for T <= 4096) or 3, + gather unless the
+    # single-CTA gate/up GEMM gathers (tensor cores, T <= 1024); FFN 2
+    # (tcgen05, plans written by the one-block dispatch), 3 (tcgen05 + plan)
+    # or 2 (CUDA cores); combine 1
+    assert L.moe_layer_launch_count(ctypes.byref(cfg())) == 1 + 1 + 2 + 1
     assert L.moe_layer_launch_count(ctypes.byref(cfg(dt=moe.MOE_F32))) == 1 + 2 + 2 + 1
-    assert L.moe_layer_launch_count(ctypes.byref(cfg(T=300))) == 2 + 2 + 3 + 1
+    assert L.moe_layer_launch_count(ctypes.byref(cfg(T=300))) == 2 + 1 + 2 + 1
+    assert L.moe_layer_launch_count(ctypes.byref(cfg(T=1100))) == 3 + 2 + 2 + 1
     big = cfg(T=16384, d=4096, N=128, Z=32, k=8, F=1024)
     assert L.moe_layer_launch_count(ctypes.byref(big)) == 3 + 4 + 3 + 1
     assert L.moe_layer_launch_count(ctypes.byref(cfg(T=0))) == 0

@@ -147,6 +147,15 @@ def run_staged_and_fused(sh: MoEShape, seed: int, sample=None, s=None):
                       d_inp.w_up, d_inp.w_down, ws, out=out2)
     torch.cuda.synchronize()
     assert torch.equal(out, out2)
+    # the fused layer equals the staged calls on the GPU's own intermediates,
+    # bit for bit; where the gate/up GEMM gathers token rows from x itself
+    # (tensor cores, T <= 1024), this pins the gather against x_perm
+    s_idx, s_gate = moe.route(ls, d_inp.x, d_inp.w_router, d_inp.bias, ws)
+    _, s_offs, _, s_slot, s_xp = moe.dispatch(ls, d_inp.x, s_idx, ws)
+    s_y = moe.expert_ffn(ls, s_xp, s_offs, d_inp.w_gate, d_inp.w_up, d_inp.w_down, ws)
+    s_out = moe.combine(ls, d_inp.x, s_y, s_idx, s_gate, s_slot)
+    torch.cuda.synchronize()
+    assert torch.equal(s_out, out), "fused layer differs from the staged calls"
     return {"flagged": int(flagged.sum()), "R": R}
 
 
