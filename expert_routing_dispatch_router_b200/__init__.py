@@ -102,6 +102,7 @@ def lib():
             "moe_layer_forward": ([C, P, P, P, P, P, P, P, P, P, sz, P], i32),
             "moe_layer_forward_host": ([C, P, P, P, P, P, P, P, P, P, sz, P], i32),
             "moe_read_device_error": ([P, P, P], i32),
+            "moe_selftest_wait_limit": ([P, ctypes.c_size_t, P], i32),
             "moe_route_noalloc": ([C, P, P, P, P, P, P, P, P], i32),
             "moe_bias_pid_update": ([C, P, P, P, ctypes.POINTER(MoEPIDParams), P], i32),
             "moe_layer_launch_count": ([C], ctypes.c_int32),
@@ -303,6 +304,14 @@ def read_device_error(ws, stream=None) -> int:
     code = ctypes.c_int32(0)
     lib().moe_read_device_error(_ptr(ws), ctypes.byref(code), _stream(stream))
     return int(code.value)
+
+
+def selftest_wait_limit(ws, stream=None) -> None:
+    """Runs the device-side wait-limit self-test: after ~2 s the workspace
+    error word holds 1 (read it with read_device_error)."""
+    _check("moe_selftest_wait_limit",
+           lib().moe_selftest_wait_limit(_ptr(ws), ws.numel() * ws.element_size(),
+                                         _stream(stream)))
 
 
 def bias_pid_update(shape: LayerShape, counts, bias, state, target: float, kp: float,

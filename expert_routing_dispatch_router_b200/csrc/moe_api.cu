@@ -300,6 +300,13 @@ moe_status_t moe_bias_pid_update(const moe_config_t* cfg, const int32_t* counts,
                                      reinterpret_cast<cudaStream_t>(stream)));
 }
 
+moe_status_t moe_selftest_wait_limit(void* ws, size_t ws_bytes, moe_stream_t stream) {
+  if (ws == nullptr || ws_bytes < 256 || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+    return MOE_ERR_WORKSPACE;
+  return cuda_status(launch_wait_limit_selftest(static_cast<int32_t*>(ws),
+                                                reinterpret_cast<cudaStream_t>(stream)));
+}
+
 moe_status_t moe_read_device_error(void* ws, int32_t* code_out, moe_stream_t stream) {
   if (ws == nullptr) return MOE_ERR_WORKSPACE;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

@@ -102,6 +102,7 @@ cudaError_t launch_bias_pid(const Shape& sh, const int32_t* counts, float* bias,
                             double* state, double target, double kp, double ki,
                             double kd, double max_step, cudaStream_t st);
 int dispatch_launch_count(const Shape& sh);
+cudaError_t launch_wait_limit_selftest(int32_t* err, cudaStream_t st);
 bool expert_ffn_uses_tensor_cores(const Shape& sh);
 int num_sms();
 

@@ -217,12 +217,21 @@ moe_status_t moe_bias_pid_update(const moe_config_t* cfg, const int32_t* counts,
 
 /* Waits for `stream`, then reads and clears the device-side error word in ws.
  * *code_out (may be NULL) gets 0 when no check failed, else a nonzero code
- * (1 = a bounded wait in the expert GEMM ran out, 2 = a routing slot held an
+ * (1 = a bounded wait in the router or an expert GEMM ran out, 2 = a routing slot held an
  * expert id outside [0, E) or one token listed an expert twice; such slots
  * are skipped). Returns
  * MOE_ERR_DEVICE_CHECK when the code is nonzero. */
 moe_status_t moe_read_device_error(void* ws, int32_t* code_out,
                                    moe_stream_t stream);
+
+/* Self-test of the device-side failure detection, for tests and health
+ * checks; it has no counterpart in the method. Launches one small kernel whose
+ * mbarrier wait can never complete. After the 2 s limit that every wait in
+ * the library has, the kernel records code 1 in the workspace error word and
+ * returns, so the context stays usable; moe_read_device_error then reports
+ * (and clears) it. Only the first 256 bytes of `ws` are used, and ws must be
+ * 256-byte aligned (else MOE_ERR_WORKSPACE). */
+moe_status_t moe_selftest_wait_limit(void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /* Number of kernel launches one moe_layer_forward call makes for cfg. */
 int32_t moe_layer_launch_count(const moe_config_t* cfg);

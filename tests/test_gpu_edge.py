@@ -1,8 +1,11 @@
 """GPU edge cases of the layer, each against the oracle or an exact property:
 T = 1, every slot on zero experts (R = 0: the expert GEMMs launch no work),
 every token on one expert, segment sizes around the 128-row token tile,
-only zero experts (N = 0), no zero experts (Z = 0), k = E, and the largest
-supported E and k."""
+only zero experts (N = 0), no zero experts (Z = 0), k = E, the largest
+supported E and k, and the device-side wait limit (a wait that nothing
+completes reports error 1 and leaves the context usable)."""
+import time
+
 import numpy as np
 import pytest
 import torch
@@ -173,3 +176,24 @@ def test_router_exact_ties_go_to_lower_id():
     np.testing.assert_array_equal(idx.cpu().numpy(), ref_idx)
     np.testing.assert_array_equal(ref_idx, np.tile(np.arange(3, 9), (sh.T, 1)))
     np.testing.assert_allclose(gate.cpu().numpy(), 1.0 / 6, rtol=1e-6)
+
+
+def test_wait_limit_reports_and_context_stays_usable():
+    # a wait that nothing completes runs out after its limit: error 1 in the
+    # workspace, read on the host; then the same context runs a layer cleanly
+    sh = MoEShape("after_timeout", T=40, d=256, n_routed=4, n_zero=2, top_k=2, ffn=256)
+    ls = moe.LayerShape(sh.T, sh.d, sh.n_routed, sh.n_zero, sh.top_k, sh.ffn)
+    ws = moe.alloc_workspace(ls)
+    t0 = time.time()
+    moe.selftest_wait_limit(ws)
+    assert moe.read_device_error(ws) == 1
+    assert 1.5 < time.time() - t0 < 30.0
+    assert moe.read_device_error(ws) == 0  # read clears it
+    inp = make_inputs(sh, 3)
+    d = inp.to("cuda")
+    out = moe.layer_forward(ls, d.x, d.w_router, d.bias, d.w_gate, d.w_up, d.w_down, ws)
+    torch.cuda.synchronize()
+    assert moe.read_device_error(ws) == 0
+    ref, _, _ = oracle.layer(inp.x, inp.w_router, inp.bias, inp.w_gate, inp.w_up, inp.w_down,
+                             sh.n_routed, sh.top_k)
+    assert out_err(out.double().cpu().numpy(), ref, inp.x.dtype) <= OUT_RTOL_RMS
