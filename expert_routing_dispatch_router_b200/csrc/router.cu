@@ -8,16 +8,21 @@
 // the bias steers selection only and that the gates are the softmax of the
 // selected raw logits (they sum to 1).
 //
-// Kernel 1 (router_logits_kernel): CUDA-core GEMM in fp32. The contraction is
-// split over blockIdx.z so that a decode batch (T ~ 64) still spreads the
-// router weights over many SMs; each split writes its partial sums to the
-// workspace and kernel 2 adds them in a fixed order, so results are
-// bit-reproducible run to run.
-//
-// Kernel 2 (topk_kernel): one warp per token. The E keys sit in registers,
-// ceil(E/32) per lane. k+1 rounds of a warp arg-max (ties to the lower id)
-// give the selection in descending key order and the margin between the k-th
-// and (k+1)-th key.
+// Three ways to the logits, all with fp32 products and sums, each followed by
+// the same warp top-k (warp_select_token):
+//  - T <= 256 (decode): router_small_kernel, one launch. TMA-staged router
+//    rows and x, FFMA partials per contraction split, and the split sums and
+//    top-k done by the last CTA of each token group.
+//  - otherwise router_logits_kernel + topk_kernel: a CUDA-core GEMM split
+//    over blockIdx.z, partials to the workspace, added in a fixed order by the
+//    top-k kernel (bit-reproducible run to run).
+//  - bf16 with T >= 512: the logits on the tensor cores from an exact
+//    three-plane bf16 split of the router weights (router_split_kernel + the
+//    grouped GEMM), then topk_kernel.
+// The top-k is one warp per token: the E keys sit in registers, ceil(E/32)
+// per lane, sorted once per lane; k+1 rounds of a warp arg-max (ties to the
+// lower id) give the selection in descending key order and the margin
+// between the k-th and (k+1)-th key.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <float.h>
