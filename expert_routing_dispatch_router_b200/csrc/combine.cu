@@ -12,6 +12,9 @@
 //
 // y_perm is fp32. Both sums run in fp32 in slot order j = 0..k-1 and the
 // result is rounded once, so the output does not depend on thread timing.
+// When the fused layer split the down GEMM's contraction (tiny batches), each
+// row of y holds ysplit partial rows, added in split order first: the same
+// arithmetic as reducing them into y_perm and combining that.
 // Grid: one block row per token, 16-byte vectors along d.
 #include "moe_internal.cuh"
 
@@ -63,7 +66,7 @@ __global__ void __launch_bounds__(128)
                    const int32_t* __restrict__ idx,
                    const float* __restrict__ gate,
                    const int32_t* __restrict__ slot_row, AT* __restrict__ out,
-                   int64_t d, int N, int k, float s) {
+                   int64_t d, int N, int k, float s, int ysplit) {
   constexpr int V = Vec<AT>::n;
   __shared__ int32_t s_row[kMaxTopK];
   __shared__ float s_gate[kMaxTopK];
@@ -97,8 +100,17 @@ __global__ void __launch_bounds__(128)
     } else {
       const int64_t r = s_row[j];
       if (r < 0) continue;
+      // y of the slot: its split partials added in order (one for plain y)
+      const float* yr = y + r * ysplit * d + col;
 #pragma unroll
-      for (int i = 0; i < V; i += 4) Vec<float>::load(y + r * d + col + i, v + i);
+      for (int i = 0; i < V; i += 4) Vec<float>::load(yr + i, v + i);
+      for (int c = 1; c < ysplit; ++c) {
+        float w[V];
+#pragma unroll
+        for (int i = 0; i < V; i += 4) Vec<float>::load(yr + (int64_t)c * d + i, w + i);
+#pragma unroll
+        for (int i = 0; i < V; ++i) v[i] += w[i];
+      }
 #pragma unroll
       for (int i = 0; i < V; ++i) racc[i] = fmaf(g, v[i], racc[i]);
     }
@@ -112,7 +124,8 @@ __global__ void __launch_bounds__(128)
 
 cudaError_t launch_combine(const Shape& sh, const void* x, const void* y_perm,
                            const int32_t* idx, const float* gate,
-                           const int32_t* slot_row, void* out, cudaStream_t st) {
+                           const int32_t* slot_row, void* out, cudaStream_t st,
+                           int ysplit) {
   const int V = sh.bf16 ? 8 : 4;
   const int64_t vecs = sh.d / V;
   const int threads = 128;
@@ -121,12 +134,12 @@ cudaError_t launch_combine(const Shape& sh, const void* x, const void* y_perm,
     launch_pdl(combine_kernel<__nv_bfloat16>, grid, dim3(threads), 0, st,
                static_cast<const __nv_bfloat16*>(x), static_cast<const float*>(y_perm),
                idx, gate, slot_row, static_cast<__nv_bfloat16*>(out), sh.d, (int)sh.N,
-               (int)sh.k, sh.s);
+               (int)sh.k, sh.s, ysplit);
   else
     launch_pdl(combine_kernel<float>, grid, dim3(threads), 0, st,
                static_cast<const float*>(x), static_cast<const float*>(y_perm), idx,
                gate, slot_row, static_cast<float*>(out), sh.d, (int)sh.N, (int)sh.k,
-               sh.s);
+               sh.s, ysplit);
   return cudaGetLastError();
 }
 

@@ -148,6 +148,12 @@ struct GemmArgs {
   // x, which reads as zeros, for the padding rows of a tile.
   const int32_t* row_token = nullptr;
   int oob_row = 0;
+  // Gate/up with a split contraction (tiny batches): when set, the epilogue
+  // writes the raw fp32 gate and up sums of split m / mt_chunk to
+  // part[row][split][0 or 1][F] (part_stride floats per row) instead of h; a
+  // fixup kernel adds the splits and applies SwiGLU.
+  float* part = nullptr;
+  int64_t part_stride = 0;
 };
 
 struct Unit {
@@ -472,7 +478,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(tempty_bar(acc));
       };
-      if (GATEUP) {
+      if (GATEUP && args.part != nullptr) {
+        const int split = un.m / args.mt_chunk;
+        float* pp = args.part + (int64_t)un.row0 * args.part_stride +
+                    (int64_t)split * 2 * args.out_cols +
+                    (int64_t)(un.m % args.mt_chunk) * BM + lrow;
+        for (int c0 = 32 * eh; c0 < un.n_mma; c0 += 64) {
+          float g[32], v[32];
+          ptx::tmem_ld32x2(tb + c0, tb + BN + c0, g, v);
+#pragma unroll
+          for (int c = 0; c < 32; ++c)
+            if (c0 + c < un.n_valid) {
+              pp[(int64_t)(c0 + c) * args.part_stride] = g[c];
+              pp[(int64_t)(c0 + c) * args.part_stride + args.out_cols] = v[c];
+            }
+        }
+        release();
+      } else if (GATEUP) {
         swiglu_epilogue<BN / 64>(tb, BN, eh, un.n_mma, un.n_valid,
                                  static_cast<__nv_bfloat16*>(args.out) + obase, args.out_cols,
                                  release);
@@ -499,6 +521,62 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// ------------------------------------- split contraction (tiny batches) --
+// h[r, f] = silu(sum_c gate_c[r, f]) * sum_c up_c[r, f] for the routed rows
+// r < R, the split partials added in order c = 0..s-1 (part as written by the
+// split gate/up epilogue: [row][c][gate | up][F] fp32).
+__global__ void __launch_bounds__(256)
+    swiglu_split_fixup_kernel(const float* __restrict__ part, int s, int64_t F,
+                              const int32_t* __restrict__ offsets, int N,
+                              __nv_bfloat16* __restrict__ h) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const int64_t R = offsets[N];
+  const int64_t fv = F / 4;
+  const int64_t stride = (int64_t)s * 2 * F;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < R * fv;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = i / fv, f = (i - r * fv) * 4;
+    const float* p = part + r * stride + f;
+    float4 g = *reinterpret_cast<const float4*>(p);
+    float4 u = *reinterpret_cast<const float4*>(p + F);
+    for (int c = 1; c < s; ++c) {
+      const float4 gc = *reinterpret_cast<const float4*>(p + (int64_t)c * 2 * F);
+      const float4 uc = *reinterpret_cast<const float4*>(p + (int64_t)c * 2 * F + F);
+      g.x += gc.x; g.y += gc.y; g.z += gc.z; g.w += gc.w;
+      u.x += uc.x; u.y += uc.y; u.z += uc.z; u.w += uc.w;
+    }
+    const __nv_bfloat162 a = __floats2bfloat162_rn(silu_f(g.x) * u.x, silu_f(g.y) * u.y);
+    const __nv_bfloat162 b = __floats2bfloat162_rn(silu_f(g.z) * u.z, silu_f(g.w) * u.w);
+    uint2 o;
+    o.x = *reinterpret_cast<const uint32_t*>(&a);
+    o.y = *reinterpret_cast<const uint32_t*>(&b);
+    *reinterpret_cast<uint2*>(h + r * F + f) = o;
+  }
+}
+
+// y[r, :] = sum_c part[r][c][:] in order c = 0..s-1, for the routed rows r < R
+// (the down GEMM's split partials, [row][c][d] fp32).
+__global__ void __launch_bounds__(256)
+    split_reduce_kernel(const float* __restrict__ part, int s, int64_t d,
+                        const int32_t* __restrict__ offsets, int N, float* __restrict__ y) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const int64_t R = offsets[N];
+  const int64_t dv = d / 4;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < R * dv;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = i / dv, col = (i - r * dv) * 4;
+    const float* p = part + r * s * d + col;
+    float4 v = *reinterpret_cast<const float4*>(p);
+    for (int c = 1; c < s; ++c) {
+      const float4 w = *reinterpret_cast<const float4*>(p + (int64_t)c * d);
+      v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
+    }
+    *reinterpret_cast<float4*>(y + r * d + col) = v;
   }
 }
 
@@ -1002,7 +1080,8 @@ bool expert_ffn_uses_tensor_cores(const Shape& sh) {
 
 int expert_ffn_launch_count(const Shape& sh) {
   if (sh.N == 0) return 0;
-  return expert_ffn_uses_tensor_cores(sh) ? 3 : 2;
+  if (!expert_ffn_uses_tensor_cores(sh)) return 2;
+  return 3 + (expert_ffn_split(sh, true) > 1 ? 1 : 0);  // plan, GEMMs, fixup
 }
 
 void expert_ffn_tiles(const Shape& sh, int* tile_gu, int* tile_dn) {
@@ -1015,12 +1094,41 @@ bool expert_ffn_gathers(const Shape& sh) {
   return expert_ffn_uses_tensor_cores(sh) && !use_pairs(sh) && tile_gateup_for(sh.T) <= 128;
 }
 
+// Contraction splits of the single-CTA expert GEMMs for tiny batches. With
+// one or a few tokens, a handful of experts gives about one 128-row unit per
+// SM, so the last units run on few SMs. Each GEMM is split so that the most
+// units the batch can have fill the SMs about four times. At most 4 splits,
+// and a divisor of the k-blocks. It stays 1 for the CTA-pair path and for
+// batches whose units already fill the SMs (decode at T = 64 among them).
+int expert_ffn_split(const Shape& sh, bool gateup) {
+  if (!expert_ffn_uses_tensor_cores(sh) || use_pairs(sh) || tile_gateup_for(sh.T) > 64)
+    return 1;
+  const int64_t experts = sh.N < sh.T * sh.k ? sh.N : sh.T * sh.k;
+  const int64_t units = experts * ((gateup ? sh.F : sh.d) / BM);
+  const int nkb = (int)((gateup ? sh.d : sh.F) / BK);
+  const int64_t want = 4ll * num_sms();
+  for (int s = 1; s <= 4; ++s)
+    if (nkb % s == 0 && units * s >= want) return s;
+  for (int s = 4; s > 1; --s)
+    if (nkb % s == 0) return s;
+  return 1;
+}
+
+int64_t expert_ffn_part_floats(const Shape& sh) {
+  const int sg = expert_ffn_split(sh, true), sd = expert_ffn_split(sh, false);
+  if (sg == 1 && sd == 1) return 0;
+  const int64_t a = sg > 1 ? (int64_t)sg * 2 * sh.F : 0;
+  const int64_t b = sd > 1 ? (int64_t)sd * sh.d : 0;
+  return sh.T * sh.k * (a > b ? a : b);
+}
+
 cudaError_t launch_expert_ffn(const Shape& sh, const void* x_perm,
                               const int32_t* offsets, const void* w_gate,
                               const void* w_up, const void* w_down, void* h,
                               void* y_perm, int32_t* tile_start, int32_t* err,
                               cudaStream_t st, const void* x_src,
-                              const int32_t* row_token, bool plan_ready) {
+                              const int32_t* row_token, bool plan_ready, float* part,
+                              bool leave_y_split) {
   if (sh.N == 0 || sh.T == 0) return cudaSuccess;
   if (!expert_ffn_uses_tensor_cores(sh)) {
     if (sh.bf16)
@@ -1085,23 +1193,45 @@ cudaError_t launch_expert_ffn(const Shape& sh, const void* x_perm,
     dp.kb_chunk = dp.num_kb;
     return launch_pair<false>(wd_map, wd_map, h16, h128, dp, st);
   }
+  // tiny batches: split contractions, fp32 partials in `part`
+  const int sg = expert_ffn_split(sh, true), sd = expert_ffn_split(sh, false);
+  if ((sg > 1 || sd > 1) && part == nullptr) return cudaErrorInvalidValue;
+  if (sg > 1) {
+    gu.m_tiles = (int)(sh.F / BM) * sg;
+    gu.kb_chunk = gu.num_kb / sg;
+    gu.part = part;
+    gu.part_stride = (int64_t)sg * 2 * sh.F;
+  }
   e = tgu == 64    ? launch_tc<true, 64>(wg_map, wu_map, x16, x128, gu, st)
       : tgu == 128 ? launch_tc<true, 128>(wg_map, wu_map, x16, x128, gu, st)
                    : launch_tc<true, 256>(wg_map, wu_map, x16, x128, gu, st);
   if (e != cudaSuccess) return e;
+  const unsigned fix_blocks = (unsigned)(2 * num_sms());
+  if (sg > 1) {
+    e = launch_pdl(swiglu_split_fixup_kernel, dim3(fix_blocks), dim3(256), 0, st,
+                   static_cast<const float*>(part), sg, sh.F, offsets, (int)sh.N,
+                   static_cast<__nv_bfloat16*>(h));
+    if (e != cudaSuccess) return e;
+  }
 
   GemmArgs dn = gu;
+  dn.row_token = nullptr;  // the down GEMM reads h, already in row order
+  dn.part = nullptr;
   dn.tile_start = tile_start + sh.N + 1;
-  dn.out = y_perm;
+  dn.out = sd > 1 ? static_cast<void*>(part) : y_perm;
   dn.num_kb = (int)(sh.F / BK);
-  dn.out_cols = (int)sh.d;
-  dn.m_tiles = (int)(sh.d / BM);
-  dn.a_rows = dn.out_cols;
-  dn.mt_chunk = dn.m_tiles;
-  dn.kb_chunk = dn.num_kb;
-  if (tdn == 64) return launch_tc<false, 64>(wd_map, wd_map, h16, h128, dn, st);
-  if (tdn == 128) return launch_tc<false, 128>(wd_map, wd_map, h16, h128, dn, st);
-  return launch_tc<false, 256>(wd_map, wd_map, h16, h128, dn, st);
+  dn.out_cols = (int)sh.d * sd;  // split c writes columns [c d, (c + 1) d)
+  dn.m_tiles = (int)(sh.d / BM) * sd;
+  dn.a_rows = (int)sh.d;
+  dn.mt_chunk = (int)(sh.d / BM);
+  dn.kb_chunk = dn.num_kb / sd;
+  e = tdn == 64    ? launch_tc<false, 64>(wd_map, wd_map, h16, h128, dn, st)
+      : tdn == 128 ? launch_tc<false, 128>(wd_map, wd_map, h16, h128, dn, st)
+                   : launch_tc<false, 256>(wd_map, wd_map, h16, h128, dn, st);
+  if (e != cudaSuccess || sd == 1 || leave_y_split) return e;
+  return launch_pdl(split_reduce_kernel, dim3(fix_blocks), dim3(256), 0, st,
+                    static_cast<const float*>(part), sd, sh.d, offsets, (int)sh.N,
+                    static_cast<float*>(y_perm));
 }
 
 }  // namespace moe

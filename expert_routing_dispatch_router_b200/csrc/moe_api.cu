@@ -44,6 +44,7 @@ WsLayout ws_layout(const Shape& sh) {
   L.x_perm = take(Tk * sh.d * sh.es);
   L.h = take(Tk * sh.F * sh.es);
   L.y_perm = take(Tk * sh.d * sizeof(float));
+  L.ffn_part = take(sh.N > 0 ? (size_t)expert_ffn_part_floats(sh) * sizeof(float) : 0);
   L.x_stage = take((size_t)sh.T * sh.d * sh.es);
   L.out_stage = take((size_t)sh.T * sh.d * sh.es);
   L.total = off;
@@ -132,11 +133,15 @@ moe_status_t run_layer(const Shape& sh, const void* x, const float* w_router,
                       slot_row, gather ? nullptr : x_perm, err, st, plan ? tile_start : nullptr,
                       tgu, tdn);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
+  // with a split down GEMM, the combine adds its partials itself
+  const int ysplit = sh.N > 0 ? expert_ffn_split(sh, false) : 1;
+  float* part = at<float>(ws, L.ffn_part);
   e = launch_expert_ffn(sh, x_perm, offsets, w_gate, w_up, w_down, at<void>(ws, L.h),
                         y_perm, tile_start, err, st, gather ? x : nullptr,
-                        gather ? row_token : nullptr, plan);
+                        gather ? row_token : nullptr, plan, part, true);
   if (e != cudaSuccess) return MOE_ERR_CUDA;
-  e = launch_combine(sh, x, y_perm, idx, gate, slot_row, out, st);
+  e = launch_combine(sh, x, ysplit > 1 ? static_cast<void*>(part) : y_perm, idx, gate,
+                     slot_row, out, st, ysplit);
   return cuda_status(e);
 }
 
@@ -211,7 +216,8 @@ moe_status_t moe_expert_ffn(const moe_config_t* cfg, const void* x_perm,
                                        at<void>(ws, L.h), y_perm,
                                        at<int32_t>(ws, L.tile_start),
                                        at<int32_t>(ws, L.header),
-                                       reinterpret_cast<cudaStream_t>(stream)));
+                                       reinterpret_cast<cudaStream_t>(stream), nullptr,
+                                       nullptr, false, at<float>(ws, L.ffn_part), false));
 }
 
 moe_status_t moe_combine(const moe_config_t* cfg, const void* x, const void* y_perm,

@@ -42,6 +42,8 @@ struct WsLayout {
   size_t x_perm;       // act   [T*k, d]
   size_t h;            // act   [T*k, F]
   size_t y_perm;       // float [T*k, d]
+  size_t ffn_part;     // float split-contraction partials of the expert GEMMs
+                       // (tiny batches only; else empty)
   size_t x_stage;      // act   [T, d]   (host-buffer entry point)
   size_t out_stage;    // act   [T, d]
   size_t total;
@@ -82,13 +84,23 @@ cudaError_t launch_expert_ffn(const Shape& sh, const void* x_perm,
                               const void* w_up, const void* w_down, void* h,
                               void* y_perm, int32_t* tile_start, int32_t* err,
                               cudaStream_t st, const void* x_src = nullptr,
-                              const int32_t* row_token = nullptr, bool plan_ready = false);
+                              const int32_t* row_token = nullptr, bool plan_ready = false,
+                              float* part = nullptr, bool leave_y_split = false);
+// Contraction splits of the expert GEMMs (1 unless the batch is tiny) and the
+// fp32 scratch they need (floats; 0 without splits). With leave_y_split the
+// down GEMM's split partials stay in `part` ([row][split][d]) for the combine
+// to add; otherwise they are added into y_perm.
+int expert_ffn_split(const Shape& sh, bool gateup);
+int64_t expert_ffn_part_floats(const Shape& sh);
 bool expert_ffn_gathers(const Shape& sh);
 // Token tiles of the gate/up and down GEMMs on the tensor-core path.
 void expert_ffn_tiles(const Shape& sh, int* tile_gu, int* tile_dn);
+// y_perm rows hold ysplit partial rows of d floats each ([row][split][d]),
+// added in split order before the gate weighting (1 for a plain y_perm).
 cudaError_t launch_combine(const Shape& sh, const void* x, const void* y_perm,
                            const int32_t* idx, const float* gate,
-                           const int32_t* slot_row, void* out, cudaStream_t st);
+                           const int32_t* slot_row, void* out, cudaStream_t st,
+                           int ysplit = 1);
 cudaError_t launch_dense_gemm_tc(const void* a, int64_t M, const void* b, int64_t T,
                                  int64_t K, int kb_chunk, float* out,
                                  const int32_t* plan, int32_t* err, cudaStream_t st);

@@ -58,8 +58,14 @@ def test_launch_count(L):
     # top-k); dispatch 1 (one block for T <= 4096) or 3, + gather unless the
     # single-CTA gate/up GEMM gathers (tensor cores, T <= 1024); FFN 2
     # (tcgen05, plans written by the one-block dispatch), 3 (tcgen05 + plan)
-    # or 2 (CUDA cores); combine 1
-    assert L.moe_layer_launch_count(ctypes.byref(cfg())) == 1 + 1 + 2 + 1
+    # or 2 (CUDA cores), + 1 SwiGLU fixup when a tiny batch splits the gate/up
+    # contraction; combine 1
+    decode = cfg(T=64, d=4096, N=128, Z=32, k=8, F=1024)
+    assert L.moe_layer_launch_count(ctypes.byref(decode)) == 1 + 1 + 2 + 1
+    # 8 experts at T=64 make 32 gate/up units: split
+    assert L.moe_layer_launch_count(ctypes.byref(cfg())) == 1 + 1 + 3 + 1
+    single = cfg(T=1, d=6144, N=256, Z=64, k=12, F=2048)
+    assert L.moe_layer_launch_count(ctypes.byref(single)) == 1 + 1 + 3 + 1
     assert L.moe_layer_launch_count(ctypes.byref(cfg(dt=moe.MOE_F32))) == 1 + 2 + 2 + 1
     assert L.moe_layer_launch_count(ctypes.byref(cfg(T=300))) == 2 + 1 + 2 + 1
     assert L.moe_layer_launch_count(ctypes.byref(cfg(T=1100))) == 3 + 2 + 2 + 1
