@@ -298,13 +298,17 @@ int dispatch_launch_count(const Shape& sh) {
   return (dispatch_small_fits(sh) ? 1 : 3) + (sh.N > 0 ? 1 : 0);
 }
 
-int num_sms() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
+int num_sms() {  // of the current device, cached per device
+  static std::atomic<int> cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  std::atomic<int>& c = cache[dev & 63];
+  int n = c.load();
+  if (n <= 0) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        n <= 0)
+      n = 148;
+    c.store(n);
   }
   return n;
 }
@@ -320,14 +324,9 @@ cudaError_t launch_dispatch(const Shape& sh, const void* x, const int32_t* idx,
   if (dispatch_small_fits(sh)) {
     const int W = (int)((sh.T + 31) / 32);
     const size_t smem = dispatch_small_smem(sh);
-    static bool attr_set = false;
-    if (!attr_set) {
-      e = cudaFuncSetAttribute(dispatch_small_kernel,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)kSmallDispatchSmem);
-      if (e != cudaSuccess) return e;
-      attr_set = true;
-    }
+    static std::atomic<uint64_t> attr_set{0};
+    e = raise_smem_once(attr_set, dispatch_small_kernel, (int)kSmallDispatchSmem);
+    if (e != cudaSuccess) return e;
     e = launch_pdl(dispatch_small_kernel, dim3(1), dim3(1024), smem, st, idx, (int)sh.T,
                    k, E, N, W, counts, offsets, row_token, slot_row, sh.T * sh.k, err,
                    tile_start, tile_gu, tile_dn);

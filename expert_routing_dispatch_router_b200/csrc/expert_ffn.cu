@@ -880,14 +880,10 @@ cudaError_t launch_tc(const CUtensorMap& a0, const CUtensorMap& a1,
                       const CUtensorMap& b16, const CUtensorMap& b128,
                       const GemmArgs& args, cudaStream_t st) {
   using C = Cfg<GATEUP, BN>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_tc_kernel<GATEUP, BN>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)C::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> attr_set{0};
+  const cudaError_t e =
+      raise_smem_once(attr_set, grouped_gemm_tc_kernel<GATEUP, BN>, (int)C::kSmemBytes);
+  if (e != cudaSuccess) return e;
   return launch_pdl(grouped_gemm_tc_kernel<GATEUP, BN>, dim3(num_sms()), dim3(kThreads),
                     C::kSmemBytes, st, a0, a1, b16, b128, args);
 }
@@ -899,12 +895,16 @@ cudaError_t launch_pair(const CUtensorMap& a0, const CUtensorMap& a1,
                         const CUtensorMap& b16, const CUtensorMap& b128,
                         const GemmArgs& args, cudaStream_t st) {
   using C = PairCfg<GATEUP>;
-  static int grid = 0;
+  static std::atomic<uint64_t> attr_set{0};
+  static std::atomic<int> grids[64];  // resident pairs x 2, per device
+  int dev = 0;
+  cudaError_t e0 = cudaGetDevice(&dev);
+  if (e0 != cudaSuccess) return e0;
+  e0 = raise_smem_once(attr_set, grouped_gemm_pair_kernel<GATEUP>, (int)C::kSmemBytes);
+  if (e0 != cudaSuccess) return e0;
+  int grid = grids[dev & 63].load();
   if (grid == 0) {
-    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_pair_kernel<GATEUP>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)C::kSmemBytes);
-    if (e != cudaSuccess) return e;
+    cudaError_t e = cudaSuccess;
     cudaLaunchConfig_t q = {};
     q.gridDim = dim3(num_sms());
     q.blockDim = dim3(kThreads);
@@ -922,6 +922,7 @@ cudaError_t launch_pair(const CUtensorMap& a0, const CUtensorMap& a1,
     if (clusters < 1) return cudaErrorInvalidConfiguration;
     const int most = num_sms() / 2;
     grid = 2 * (clusters < most ? clusters : most);
+    grids[dev & 63].store(grid);
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);

@@ -6,6 +6,7 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <utility>
 
 #include "../../include/moe_api.h"
@@ -117,6 +118,22 @@ int dispatch_launch_count(const Shape& sh);
 cudaError_t launch_wait_limit_selftest(int32_t* err, cudaStream_t st);
 bool expert_ffn_uses_tensor_cores(const Shape& sh);
 int num_sms();
+
+// Raises a kernel's dynamic shared-memory limit once per device (the
+// attribute is per device; one process may drive several GPUs). `done` is the
+// calling launcher's set of devices already done; racing threads only repeat
+// the idempotent call.
+template <typename Kernel>
+cudaError_t raise_smem_once(std::atomic<uint64_t>& done, Kernel kernel, int bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = 1ull << (dev & 63);
+  if (done.load() & bit) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.fetch_or(bit);
+  return e;
+}
 
 // Launch with programmatic dependent launch allowed: the kernel may start
 // while its predecessor on the stream drains, and must call griddep_wait()

@@ -739,18 +739,9 @@ cudaError_t launch_small(dim3 grid, size_t smem, cudaStream_t st, const CUtensor
                          const CUtensorMap& tm_x, const float* bias, float* part, int32_t* counter, int32_t* err,
                          float* logits_out, int32_t* idx, float* gate, uint8_t* flags, int T,
                          int d, int E, int k, int ksplit) {
-  // the shared-memory limit is raised once per device and instantiation
   static std::atomic<uint64_t> attr_set{0};
-  int dev = 0;
-  cudaError_t a = cudaGetDevice(&dev);
+  const cudaError_t a = raise_smem_once(attr_set, router_small_kernel<XT, PL>, kSmallMaxBytes);
   if (a != cudaSuccess) return a;
-  const uint64_t bit = 1ull << (dev & 63);
-  if (!(attr_set.load() & bit)) {
-    a = cudaFuncSetAttribute(router_small_kernel<XT, PL>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, kSmallMaxBytes);
-    if (a != cudaSuccess) return a;
-    attr_set.fetch_or(bit);
-  }
   return launch_pdl(router_small_kernel<XT, PL>, grid, dim3(256), smem, st, tm_w, tm_x, bias,
                     part, counter, err, logits_out, idx, gate, flags, T, d, E, k, ksplit);
 }
