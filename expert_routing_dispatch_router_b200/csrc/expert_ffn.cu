@@ -478,7 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(tempty_bar(acc));
       };
-      if (GATEUP && args.part != nullptr) {
+      if (GATEUP && BN == 64 && args.part != nullptr) {  // splits only at T <= 64
         const int split = un.m / args.mt_chunk;
         float* pp = args.part + (int64_t)un.row0 * args.part_stride +
                     (int64_t)split * 2 * args.out_cols +
