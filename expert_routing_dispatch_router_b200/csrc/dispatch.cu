@@ -239,7 +239,11 @@ __global__ void __launch_bounds__(1024)
     __syncthreads();
     const int32_t dn = block_exclusive_scan((v + tile_dn - 1) / tile_dn, warp_sums, &tot);
     if ((int)threadIdx.x < N) tile_start[N + 1 + threadIdx.x] = dn;
-    if (threadIdx.x == 0) tile_start[2 * N + 1] = tot;
+    if (threadIdx.x == 0) {
+      tile_start[2 * N + 1] = tot;
+      tile_start[2 * N + 2] = 0;  // the CTA-pair GEMMs' unit counters
+      tile_start[2 * N + 3] = 0;
+    }
     __syncthreads();
   }
   for (int t = threadIdx.x; t < T; t += blockDim.x) {

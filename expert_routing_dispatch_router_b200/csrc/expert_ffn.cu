@@ -90,6 +90,10 @@ __global__ void __launch_bounds__(1024)
   griddep_launch_dependents();
   tile_prefix(offsets, N, tile_gu, tile_start, warp_sums);
   tile_prefix(offsets, N, tile_dn, tile_start + N + 1, warp_sums);
+  if (threadIdx.x == 0) {  // the CTA-pair GEMMs' unit counters
+    tile_start[2 * N + 2] = 0;
+    tile_start[2 * N + 3] = 0;
+  }
 }
 
 // ------------------------------------------------------- tensor-core path --
@@ -99,6 +103,10 @@ constexpr int BK = 64;   // contraction elements per stage: 128-byte rows
 // per TMEM lane quarter, splitting the accumulator columns)
 constexpr int kThreads = 320;
 constexpr int kEpiWarps = 8;
+// CTA pairs: unit ring depth and readers of each slot (leader MMA thread,
+// leader epilogue warps, peer producer, peer epilogue warps)
+constexpr int kRing = 4;
+constexpr int kRingReaders = 1 + kEpiWarps + 1 + kEpiWarps;
 constexpr uint32_t kTileBytes = BM * BK * 2;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccStride = 256;  // TMEM columns per accumulator buffer (2 buffers)
@@ -154,6 +162,9 @@ struct GemmArgs {
   // fixup kernel adds the splits and applies SwiGLU.
   float* part = nullptr;
   int64_t part_stride = 0;
+  // CTA pairs: units are handed out in order from this counter (zeroed with
+  // the tile plan before the launch)
+  int* unit_counter = nullptr;
 };
 
 struct Unit {
@@ -197,6 +208,24 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity,
   while (true) {
     for (int i = 0; i < 64; ++i)
       if (ptx::mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (ptx::global_timer_ns() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      atomicCAS(err, 0, kErrWaitTimeout);
+      return false;
+    }
+  }
+}
+
+// wait_bounded with cluster-scope acquire (phases completed by the other CTA).
+__device__ __forceinline__ bool wait_bounded_cluster(uint32_t bar, uint32_t parity,
+                                                     volatile int* abort_flag,
+                                                     int32_t* err) {
+  if (ptx::mbar_try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = ptx::global_timer_ns();
+  while (true) {
+    for (int i = 0; i < 64; ++i)
+      if (ptx::mbar_try_wait_cluster(bar, parity)) return true;
     if (*abort_flag) return false;
     if (ptx::global_timer_ns() - t0 > kWaitLimitNs) {
       *abort_flag = 1;
@@ -638,6 +667,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t mma_done_bar = bars + 8u * (2 * S + 4);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + 8 * (2 * S + 5));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  // unit ring: the leader's producer hands each unit id to both CTAs
+  auto ring_full = [&](int r) { return bars + 160u + 8u * r; };
+  auto ring_empty = [&](int r) { return bars + 192u + 8u * r; };
+  volatile int* s_ring = reinterpret_cast<volatile int*>(smem + C::kBarOff + 224);
   int* s_tiles = reinterpret_cast<int*>(smem + C::kTabOff);
   int* s_offs = s_tiles + (kMaxExperts + 1);
 
@@ -645,7 +678,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int N = args.N;
   const uint32_t rank = ptx::cluster_ctarank();
   const bool leader = rank == 0;
-  const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       ptx::mbar_init(full_bar(s), 1);
@@ -656,6 +688,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::mbar_init(tempty_bar(b), 2 * kEpiWarps);
     }
     ptx::mbar_init(mma_done_bar, 1);
+    for (int r = 0; r < kRing; ++r) {
+      ptx::mbar_init(ring_full(r), 1);
+      ptx::mbar_init(ring_empty(r), kRingReaders);
+    }
     *abort_flag = 0;
     ptx::fence_mbar_init();
   }
@@ -681,6 +717,34 @@ __global__ void __launch_bounds__(kThreads, 1)
   ptx::tc_fence_after();
   const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
   const int total_units = s_tiles[N] * args.m_tiles;
+  // Dynamic schedule: the leader's producer takes the next unit from the
+  // global counter (-1 once none are left) and publishes it in ring slot
+  // seq % kRing of both CTAs; every other role reads its units from there, in
+  // the same order. A slot is reused once its kRingReaders readers (the
+  // leader's MMA thread and epilogue warps, the peer's producer and epilogue
+  // warps) have arrived on the leader's ring_empty.
+  auto publish = [&](int seq, int u) -> bool {
+    const int r = seq % kRing;
+    const uint32_t par = (uint32_t)(seq / kRing) & 1u;
+    if (!wait_bounded(ring_empty(r), par ^ 1u, abort_flag, args.err)) return false;
+    s_ring[r] = u;
+    ptx::st_shared_cluster_u32(ptx::map_to_rank(ptx::smem_addr((const void*)(s_ring + r)), 1),
+                               (uint32_t)u);
+    ptx::mbar_arrive(ring_full(r));
+    ptx::mbar_arrive_remote(ptx::map_to_rank(ring_full(r), 1));
+    return true;
+  };
+  auto take = [&](int seq, int* u) -> bool {
+    const int r = seq % kRing;
+    const uint32_t par = (uint32_t)(seq / kRing) & 1u;
+    if (!wait_bounded_cluster(ring_full(r), par, abort_flag, args.err)) return false;
+    *u = s_ring[r];
+    if (leader)
+      ptx::mbar_arrive(ring_empty(r));
+    else
+      ptx::mbar_arrive_remote(ptx::map_to_rank(ring_empty(r), 0));
+    return true;
+  };
 
   if (warp == 0) {
     // ---------------------------------------------------- TMA producer --
@@ -691,7 +755,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0, armed = 0, armed_par = 0;
       bool ok = true, issued = false;
-      for (int u = cid; u < total_units && ok; u += ncl) {
+      for (int seq = 0; ok; ++seq) {
+        int u = -1;
+        if (leader) {
+          u = atomicAdd(args.unit_counter, 1);
+          if (u >= total_units) u = -1;
+          ok = publish(seq, u);
+        } else {
+          ok = take(seq, &u);
+        }
+        if (!ok || u < 0) break;
         const Unit un = decode_unit<BN>(u, s_tiles, s_offs, N, args.m_tiles);
         const int n_pair = (un.n_valid + 31) & ~31;  // MMA N; each CTA holds half
         const int half = n_pair >> 1;
@@ -742,7 +815,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true, issued = false;
-      for (int u = cid; u < total_units && ok; u += ncl) {
+      for (int seq = 0; ok; ++seq) {
+        int u = -1;
+        ok = take(seq, &u);
+        if (!ok || u < 0) break;
         const Unit un = decode_unit<BN>(u, s_tiles, s_offs, N, args.m_tiles);
         const int n_pair = (un.n_valid + 31) & ~31;
         if (!wait_bounded(tempty_bar(acc), acc_phase ^ 1u, abort_flag, args.err)) {
@@ -795,7 +871,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int lrow = ew * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int u = cid; u < total_units; u += ncl) {
+    for (int seq = 0;; ++seq) {
+      int u = -1;
+      bool got = true;
+      if (lane == 0) got = take(seq, &u);
+      got = __shfl_sync(0xffffffffu, got, 0);
+      u = __shfl_sync(0xffffffffu, u, 0);
+      if (!got || u < 0) break;
       const Unit un = decode_unit<BN>(u, s_tiles, s_offs, N, args.m_tiles);
       const int n_pair = (un.n_valid + 31) & ~31;
       const bool ok = wait_bounded(tfull_bar(acc), acc_phase, abort_flag, args.err);
@@ -1181,9 +1263,12 @@ cudaError_t launch_expert_ffn(const Shape& sh, const void* x_perm,
   if (pairs) {
     GemmArgs gp = gu;
     gp.m_tiles = (int)(sh.F / 256);  // pairs of 128-row tiles
+    gp.unit_counter = tile_start + 2 * sh.N + 2;
     e = launch_pair<true>(wg_map, wu_map, x16, x128, gp, st);
     if (e != cudaSuccess) return e;
     GemmArgs dp = gu;
+    dp.row_token = nullptr;  // the down GEMM reads h, already in row order
+    dp.unit_counter = tile_start + 2 * sh.N + 3;
     dp.tile_start = tile_start + sh.N + 1;
     dp.out = y_perm;
     dp.num_kb = (int)(sh.F / BK);

@@ -40,7 +40,7 @@ WsLayout ws_layout(const Shape& sh) {
   L.offsets = take((size_t)(sh.N + 1) * sizeof(int32_t));
   L.row_token = take(Tk * sizeof(int32_t));
   L.slot_row = take(Tk * sizeof(int32_t));
-  L.tile_start = take(2 * (size_t)(sh.N + 1) * sizeof(int32_t));
+  L.tile_start = take((2 * (size_t)(sh.N + 1) + 2) * sizeof(int32_t));
   L.x_perm = take(Tk * sh.d * sh.es);
   L.h = take(Tk * sh.F * sh.es);
   L.y_perm = take(Tk * sh.d * sizeof(float));

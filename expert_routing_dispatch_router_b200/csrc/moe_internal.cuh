@@ -39,7 +39,8 @@ struct WsLayout {
   size_t offsets;      // int32 [N + 1]
   size_t row_token;    // int32 [T*k]
   size_t slot_row;     // int32 [T*k]
-  size_t tile_start;   // int32 [2 (N + 1)] (expert GEMM plans)
+  size_t tile_start;   // int32 [2 (N + 1) + 2]: the expert GEMMs' plans, then
+                       // the CTA-pair GEMMs' unit counters
   size_t x_perm;       // act   [T*k, d]
   size_t h;            // act   [T*k, F]
   size_t y_perm;       // float [T*k, d]
