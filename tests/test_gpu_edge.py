@@ -73,10 +73,33 @@ def test_all_tokens_to_one_expert_multiple_tiles():
     assert counts[2] == 300
 
 
+PAIRS = MoEShape("pairs_edge", T=1100, d=512, n_routed=6, n_zero=2, top_k=2, ffn=512)
+
+
+def test_pairs_all_tokens_to_one_expert():
+    # T > 1024: CTA pairs; one expert gets every token (9 token tiles x 2
+    # weight tiles, all taken from the unit counter by whichever pair is free)
+    inp = make_inputs(PAIRS, 12)
+    inp.bias[3] += 1e3
+    out, counts = check_layer(PAIRS, inp)
+    assert counts[3] == PAIRS.T
+
+
+def test_pairs_no_routed_slots():
+    # CTA pairs with no work at all: the first unit handed out is the end mark
+    inp = make_inputs(PAIRS, 13)
+    inp.bias[PAIRS.n_routed:] += 1e3
+    out, counts = fused(PAIRS, inp)
+    assert counts[: PAIRS.n_routed].sum() == 0
+    diff = (out.float() - inp.x.float()).abs()
+    assert float((diff / inp.x.float().abs().clamp_min(1e-30)).max()) <= 2 ** -8
+
+
 @pytest.mark.parametrize("sizes,F", [((1, 127, 128, 129, 0, 256, 3), 384),
                                      ((255, 0, 0, 1, 17, 384, 64), 384),
                                      # T > 1024: both GEMMs run on CTA pairs
-                                     ((1, 31, 32, 33, 255, 256, 257, 300), 512)])
+                                     ((1, 31, 32, 33, 255, 256, 257, 300), 512),
+                                     ((0, 600, 0, 1, 520), 512)])
 def test_expert_segments_around_tile_size(sizes, F):
     """moe_expert_ffn on crafted segments: offsets give exactly these rows per
     expert; rows are random bf16; checked row by row against the oracle."""
