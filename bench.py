@@ -191,9 +191,23 @@ def cpu_baseline(sh, inp, budget_s=12.0):
         if time.perf_counter() - t0 >= budget_s or done >= 64 * n_tok:
             break
     dt = time.perf_counter() - t0
+    # the same on one core, on a few tokens (about 3 s)
+    n1 = min(n_tok, 4)
+    oracle.set_num_threads(1)
+    try:
+        done1, t1 = 0, time.perf_counter()
+        while done1 == 0 or (time.perf_counter() - t1 < 3.0 and done1 < 64 * n1):
+            oracle.layer(inp.x, inp.w_router, inp.bias, inp.w_gate, inp.w_up, inp.w_down,
+                         sh.n_routed, sh.top_k, sh.routed_scale, tokens=toks[:n1])
+            done1 += n1
+        dt1 = time.perf_counter() - t1
+    finally:
+        oracle.set_num_threads(cores)
     return {"value": done / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
             "sample": f"whole layer (fp64) on {n_tok} of {sh.T} tokens, repeated "
-                      f"{done // n_tok}x ({dt:.1f} s)"}
+                      f"{done // n_tok}x ({dt:.1f} s)",
+            "single_core": {"value": done1 / dt1, "unit": "tokens/s",
+                            "sample": f"{n1} tokens, repeated {done1 // n1}x ({dt1:.1f} s)"}}
 
 
 # -------------------------------------------------------------- GPU path --
@@ -364,15 +378,30 @@ def run_gpu(args, sh):
         n_zero_tok = int(((idx >= sh.n_routed).any(dim=1)).sum())
         b_comb = R * sh.d * 4 + n_zero_tok * sh.d * es + sh.T * sh.d * es + Tk * 12
         flops_ffn = 6.0 * R * sh.d * sh.ffn
+        hbm = pk["hbm_gbs"]
+
+        def gbs(b, ms):
+            g = b / ms / 1e6
+            return {"ms": ms, "gbs": g, "frac_of_measured_hbm": g / hbm,
+                    "frac_of_8tbs": g / 8000.0}
+
+        flops_router = 2.0 * sh.T * sh.d * sh.E
+        # whole layer against its own ceiling: the larger of its FLOPs at the
+        # bf16 peak and its algorithmic bytes at the HBM peak
+        b_layer = b_route + b_ffn + sh.T * sh.d * es * 2
+        t_floor_ms = max((flops_ffn + flops_router) / (pk["bf16_tflops"] * 1e9),
+                         b_layer / (hbm * 1e6))
         comp = {
-            "router_topk": {"ms": t_route, "gbs": b_route / t_route / 1e6},
-            "dispatch": {"ms": t_disp, "gbs": b_disp / t_disp / 1e6},
+            "router_topk": gbs(b_route, t_route),
+            "dispatch": gbs(b_disp, t_disp),
             "expert_ffn": {"ms": t_ffn, "gbs": b_ffn / t_ffn / 1e6,
                            "tflops": flops_ffn / t_ffn / 1e9,
                            "tensor_frac_of_measured_bf16": flops_ffn / t_ffn / 1e9
-                           / pk["bf16_tflops"]},
-            "combine": {"ms": t_comb, "gbs": b_comb / t_comb / 1e6},
-            "layer_graph": {"ms": t_graph, "tokens_per_s": sh.T / (t_graph / 1e3)},
+                           / pk["bf16_tflops"],
+                           "tensor_frac_of_2250_spec": flops_ffn / t_ffn / 1e9 / 2250.0},
+            "combine": gbs(b_comb, t_comb),
+            "layer_graph": {"ms": t_graph, "tokens_per_s": sh.T / (t_graph / 1e3),
+                            "roofline_frac": t_floor_ms / t_graph},
             "R": R, "U": U,
         }
         # the bound is whichever ceiling is lower for this batch: weight bytes
