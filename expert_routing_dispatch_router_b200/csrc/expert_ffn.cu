@@ -1132,7 +1132,7 @@ cudaError_t launch_simt(const Shape& sh, const void* x_perm, const int32_t* offs
 // (fp32, bf16 inputs). M is a multiple of 128 and K of kb_chunk * 64. Every
 // chunk starts a fresh accumulator, which bounds the accumulation chain the
 // tensor cores' fp32 adder runs through. plan is a device int32[4] holding
-// {0, T, 0, ceil(T / kTileDown)} (the expert's rows, then its token tiles).
+// {0, T, 0, ceil(T / kRouterGemmTile)} (the expert's rows, then its token tiles).
 cudaError_t launch_dense_gemm_tc(const void* a, int64_t M, const void* b, int64_t T,
                                  int64_t K, int kb_chunk, float* out,
                                  const int32_t* plan, int32_t* err, cudaStream_t st) {
@@ -1154,7 +1154,7 @@ cudaError_t launch_dense_gemm_tc(const void* a, int64_t M, const void* b, int64_
   g.a_rows = (int)M;
   g.mt_chunk = (int)(M / BM);
   g.kb_chunk = kb_chunk;
-  return launch_tc<false, kTileDown>(am, am, b16, b128, g, st);
+  return launch_tc<false, kRouterGemmTile>(am, am, b16, b128, g, st);
 }
 
 bool expert_ffn_uses_tensor_cores(const Shape& sh) {

@@ -16,8 +16,7 @@ namespace moe {
 constexpr int kMaxExperts = 1024;  // top-k keeps E/32 keys per lane
 constexpr int kMaxTopK = 32;       // one gate per lane
 constexpr int kChunkTokens = 256;  // tokens per dispatch block
-constexpr int kTileGateUp = 128;   // token tile of the gate/up expert GEMM
-constexpr int kTileDown = 256;     // token tile of the down expert GEMM
+constexpr int kRouterGemmTile = 256;  // token tile of the tensor-core router GEMM
 constexpr int kWsAlign = 1024;
 
 // Device error codes written into the workspace header.

@@ -790,7 +790,7 @@ cudaError_t launch_router(const Shape& sh, const void* x, const float* w_r,
     if (blocks > 4 * num_sms()) blocks = 4 * num_sms();
     e = launch_pdl(router_split_kernel, dim3((unsigned)blocks), dim3(256), 0, st,
                    reinterpret_cast<const float4*>(w_r), sh.E, sh.d, Ep,
-                   static_cast<uint2*>(planes), plan, sh.T, kTileDown);
+                   static_cast<uint2*>(planes), plan, sh.T, kRouterGemmTile);
     if (e != cudaSuccess) return e;
     e = launch_dense_gemm_tc(planes, Ep, x, sh.T, sh.d, router_kb_chunk(sh), part, plan,
                              err, st);
