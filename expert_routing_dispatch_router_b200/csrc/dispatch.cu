@@ -194,19 +194,22 @@ __global__ void __launch_bounds__(1024)
   __shared__ int32_t warp_sums[32];
   griddep_wait();
   griddep_launch_dependents();
+  // one thread per routing slot s (token s / k): every slot's expert id is
+  // one load, and a thread's first slot stays in a register for the ranks
+  const int Tk = T * k;
+  const int e_first = (int)threadIdx.x < Tk ? idx[threadIdx.x] : -1;
   for (int i = threadIdx.x; i < E * W; i += blockDim.x) mask[i] = 0u;
   __syncthreads();
-  for (int t = threadIdx.x; t < T; t += blockDim.x) {
-    const uint32_t bit = 1u << (t & 31);
-    for (int j = 0; j < k; ++j) {
-      const int e = idx[(int64_t)t * k + j];
-      if (e < 0 || e >= E) {
-        record_error(err, kErrBadExpertId);
-        continue;
-      }
-      const uint32_t old = atomicOr(&mask[e * W + (t >> 5)], bit);
-      if (old & bit) record_error(err, kErrBadExpertId);
+  for (int s = threadIdx.x; s < Tk; s += blockDim.x) {
+    const int e = s == (int)threadIdx.x ? e_first : idx[s];
+    const int t = s / k;
+    if (e < 0 || e >= E) {
+      record_error(err, kErrBadExpertId);
+      continue;
     }
+    const uint32_t bit = 1u << (t & 31);
+    const uint32_t old = atomicOr(&mask[e * W + (t >> 5)], bit);
+    if (old & bit) record_error(err, kErrBadExpertId);
   }
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
@@ -246,18 +249,16 @@ __global__ void __launch_bounds__(1024)
     }
     __syncthreads();
   }
-  for (int t = threadIdx.x; t < T; t += blockDim.x) {
+  for (int s = threadIdx.x; s < Tk; s += blockDim.x) {
+    const int e = s == (int)threadIdx.x ? e_first : idx[s];
+    const int t = s / k;
     const int w = t >> 5;
-    const uint32_t below = (1u << (t & 31)) - 1u;
-    for (int j = 0; j < k; ++j) {
-      const int e = idx[(int64_t)t * k + j];
-      int32_t r = -1;
-      if (e >= 0 && e < N) {
-        r = s_off[e] + pre[e * W + w] + __popc(mask[e * W + w] & below);
-        row_token[r] = t;
-      }
-      slot_row[(int64_t)t * k + j] = r;
+    int32_t r = -1;
+    if (e >= 0 && e < N) {
+      r = s_off[e] + pre[e * W + w] + __popc(mask[e * W + w] & ((1u << (t & 31)) - 1u));
+      row_token[r] = t;
     }
+    slot_row[s] = r;
   }
   for (int64_t r = R + threadIdx.x; r < rows_cap; r += blockDim.x) row_token[r] = -1;
 }
