@@ -86,33 +86,50 @@ __global__ void __launch_bounds__(128)
   float racc[V], zacc[V], v[V];
 #pragma unroll
   for (int i = 0; i < V; ++i) racc[i] = zacc[i] = 0.f;
-  bool have_x = false;
+  bool have_zero = false;
+  for (int j = 0; j < k; ++j) have_zero |= s_zero[j] != 0;
   float xv[V];
-  for (int j = 0; j < k; ++j) {
-    const float g = s_gate[j];
-    if (s_zero[j]) {
-      if (!have_x) {
-        Vec<AT>::load(x + t * d + col, xv);
-        have_x = true;
+  if (have_zero) Vec<AT>::load(x + t * d + col, xv);
+  // slots four at a time: the y loads of a group are issued together, then
+  // added in slot order
+  for (int j0 = 0; j0 < k; j0 += 4) {
+    const float* yr[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int j = j0 + q;
+      const int r = j < k && !s_zero[j] ? s_row[j] : -1;
+      yr[q] = r >= 0 ? y + (int64_t)r * ysplit * d + col : nullptr;
+    }
+    float yv[4][V];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (yr[q] != nullptr) {
+#pragma unroll
+        for (int i = 0; i < V; i += 4) Vec<float>::load(yr[q] + i, yv[q] + i);
       }
+    // split partials of each slot's row, added in split order (none for plain y)
+    for (int c = 1; c < ysplit; ++c) {
 #pragma unroll
-      for (int i = 0; i < V; ++i) zacc[i] = fmaf(g, xv[i], zacc[i]);
-    } else {
-      const int64_t r = s_row[j];
-      if (r < 0) continue;
-      // y of the slot: its split partials added in order (one for plain y)
-      const float* yr = y + r * ysplit * d + col;
+      for (int q = 0; q < 4; ++q)
+        if (yr[q] != nullptr) {
 #pragma unroll
-      for (int i = 0; i < V; i += 4) Vec<float>::load(yr + i, v + i);
-      for (int c = 1; c < ysplit; ++c) {
-        float w[V];
+          for (int i = 0; i < V; i += 4) Vec<float>::load(yr[q] + (int64_t)c * d + i, v + i);
 #pragma unroll
-        for (int i = 0; i < V; i += 4) Vec<float>::load(yr + (int64_t)c * d + i, w + i);
+          for (int i = 0; i < V; ++i) yv[q][i] += v[i];
+        }
+    }
 #pragma unroll
-        for (int i = 0; i < V; ++i) v[i] += w[i];
+    for (int q = 0; q < 4; ++q) {
+      const int j = j0 + q;
+      if (j >= k) continue;
+      const float g = s_gate[j];
+      if (s_zero[j]) {
+#pragma unroll
+        for (int i = 0; i < V; ++i) zacc[i] = fmaf(g, xv[i], zacc[i]);
+      } else if (yr[q] != nullptr) {
+#pragma unroll
+        for (int i = 0; i < V; ++i) racc[i] = fmaf(g, yv[q][i], racc[i]);
       }
-#pragma unroll
-      for (int i = 0; i < V; ++i) racc[i] = fmaf(g, v[i], racc[i]);
     }
   }
 #pragma unroll
