@@ -167,11 +167,11 @@ moe_status_t moe_route(const moe_config_t* cfg, const void* x, const float* w_ro
   Shape sh;
   moe_status_t s = make_shape(cfg, &sh);
   if (s != MOE_OK) return s;
+  if (sh.T == 0) return MOE_OK;  // empty batch: nothing is read or written
   if (!dev_ok(x) || !dev_ok(w_router) || !dev_ok(bias) || !dev_ok(topk_idx) ||
       !dev_ok(topk_gate) || !opt_ok(logits) || !opt_ok(flags))
     return MOE_ERR_INVALID_ARG;
   if ((s = check_ws(sh, ws, ws_bytes)) != MOE_OK) return s;
-  if (sh.T == 0) return MOE_OK;
   const WsLayout L = ws_layout(sh);
   return cuda_status(launch_router(sh, x, w_router, bias, at<float>(ws, L.logits),
                                    topk_idx, topk_gate, flags, logits,
@@ -187,11 +187,11 @@ moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t*
   Shape sh;
   moe_status_t s = make_shape(cfg, &sh);
   if (s != MOE_OK) return s;
+  if (sh.T == 0) return MOE_OK;  // empty batch: nothing is read or written
   if (!dev_ok(x) || !dev_ok(topk_idx) || !dev_ok(counts) || !dev_ok(offsets) ||
       !dev_ok(row_token) || !dev_ok(slot_row) || !dev_ok(x_perm))
     return MOE_ERR_INVALID_ARG;
   if ((s = check_ws(sh, ws, ws_bytes)) != MOE_OK) return s;
-  if (sh.T == 0) return MOE_OK;
   const WsLayout L = ws_layout(sh);
   return cuda_status(launch_dispatch(sh, x, topk_idx, at<int32_t>(ws, L.chunk_base),
                                      counts, offsets, row_token, slot_row, x_perm,
@@ -206,11 +206,11 @@ moe_status_t moe_expert_ffn(const moe_config_t* cfg, const void* x_perm,
   Shape sh;
   moe_status_t s = make_shape(cfg, &sh);
   if (s != MOE_OK) return s;
+  if (sh.T == 0) return MOE_OK;  // empty batch: nothing is read or written
   if (!dev_ok(x_perm) || !dev_ok(offsets) || !dev_ok(y_perm)) return MOE_ERR_INVALID_ARG;
   if (sh.N > 0 && (!dev_ok(w_gate) || !dev_ok(w_up) || !dev_ok(w_down)))
     return MOE_ERR_INVALID_ARG;
   if ((s = check_ws(sh, ws, ws_bytes)) != MOE_OK) return s;
-  if (sh.T == 0) return MOE_OK;
   const WsLayout L = ws_layout(sh);
   return cuda_status(launch_expert_ffn(sh, x_perm, offsets, w_gate, w_up, w_down,
                                        at<void>(ws, L.h), y_perm,
@@ -226,10 +226,10 @@ moe_status_t moe_combine(const moe_config_t* cfg, const void* x, const void* y_p
   Shape sh;
   moe_status_t s = make_shape(cfg, &sh);
   if (s != MOE_OK) return s;
+  if (sh.T == 0) return MOE_OK;  // empty batch: nothing is read or written
   if (!dev_ok(x) || !dev_ok(y_perm) || !dev_ok(topk_idx) || !dev_ok(topk_gate) ||
       !dev_ok(slot_row) || !dev_ok(out))
     return MOE_ERR_INVALID_ARG;
-  if (sh.T == 0) return MOE_OK;
   return cuda_status(launch_combine(sh, x, y_perm, topk_idx, topk_gate, slot_row, out,
                                     reinterpret_cast<cudaStream_t>(stream)));
 }
@@ -242,13 +242,13 @@ moe_status_t moe_layer_forward(const moe_config_t* cfg, const void* x,
   Shape sh;
   moe_status_t s = make_shape(cfg, &sh);
   if (s != MOE_OK) return s;
+  if (sh.T == 0) return MOE_OK;  // empty batch: nothing is read or written
   if (!dev_ok(x) || !dev_ok(w_router) || !dev_ok(bias) || !dev_ok(out) ||
       !opt_ok(counts))
     return MOE_ERR_INVALID_ARG;
   if (sh.N > 0 && (!dev_ok(w_gate) || !dev_ok(w_up) || !dev_ok(w_down)))
     return MOE_ERR_INVALID_ARG;
   if ((s = check_ws(sh, ws, ws_bytes)) != MOE_OK) return s;
-  if (sh.T == 0) return MOE_OK;
   return run_layer(sh, x, w_router, bias, w_gate, w_up, w_down, out, counts, ws,
                    reinterpret_cast<cudaStream_t>(stream));
 }
@@ -262,12 +262,12 @@ moe_status_t moe_layer_forward_host(const moe_config_t* cfg, const void* x_host,
   Shape sh;
   moe_status_t s = make_shape(cfg, &sh);
   if (s != MOE_OK) return s;
+  if (sh.T == 0) return MOE_OK;  // empty batch: nothing is read or written
   if (x_host == nullptr || out_host == nullptr || !dev_ok(w_router) || !dev_ok(bias))
     return MOE_ERR_INVALID_ARG;
   if (sh.N > 0 && (!dev_ok(w_gate) || !dev_ok(w_up) || !dev_ok(w_down)))
     return MOE_ERR_INVALID_ARG;
   if ((s = check_ws(sh, ws, ws_bytes)) != MOE_OK) return s;
-  if (sh.T == 0) return MOE_OK;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const WsLayout L = ws_layout(sh);
   const size_t act_bytes = (size_t)sh.T * sh.d * sh.es;

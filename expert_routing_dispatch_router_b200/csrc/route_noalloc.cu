@@ -70,12 +70,12 @@ extern "C" moe_status_t moe_route_noalloc(const moe_config_t* cfg, const void* x
   Shape sh;
   const moe_status_t s = shape_from_config(cfg, &sh);  // the checks of every call
   if (s != MOE_OK) return s;
+  if (sh.T == 0) return MOE_OK;  // empty batch: nothing is read or written
   if (x == nullptr || w_router == nullptr || bias == nullptr || topk_idx == nullptr ||
       topk_gate == nullptr || !aligned16(x) || !aligned16(w_router) || !aligned16(bias) ||
       !aligned16(topk_idx) || !aligned16(topk_gate) || !aligned16(logits) ||
       !aligned16(flags))
     return MOE_ERR_INVALID_ARG;
-  if (sh.T == 0) return MOE_OK;
   // the partial sums of one split need T * E floats
   const int64_t per_split = sh.T * sh.E;
   if (per_split > kNoAllocScratchFloats) return MOE_ERR_UNSUPPORTED;

@@ -663,7 +663,8 @@ int small_chunk_bytes(const Shape& sh) {
 }
 
 int router_small_plan(const Shape& sh, int* ksplit_out) {
-  const int64_t base = ((sh.T + DG - 1) / DG) * ((sh.E + DE - 1) / DE);
+  int64_t base = ((sh.T + DG - 1) / DG) * ((sh.E + DE - 1) / DE);
+  if (base < 1) base = 1;  // an empty batch still gets a valid plan
   int64_t chunks = (kSmallMaxBytes - kSmallHeader) / small_chunk_bytes(sh);
   if (chunks > kSmallMaxChunks) chunks = kSmallMaxChunks;
   const int64_t kmax = chunks * kSmallChunk;
@@ -687,7 +688,8 @@ int router_launch_count(const Shape& sh) {
 
 // Number of contraction splits so that the logits GEMM has >= ~2 CTAs per SM.
 int router_splits(const Shape& sh) {
-  const int64_t tiles = ((sh.E + RE - 1) / RE) * ((sh.T + RT - 1) / RT);
+  int64_t tiles = ((sh.E + RE - 1) / RE) * ((sh.T + RT - 1) / RT);
+  if (tiles < 1) tiles = 1;  // an empty batch still gets a valid plan
   int64_t want = (2 * num_sms() + tiles - 1) / tiles;
   int64_t max_split = (sh.d + 255) / 256;  // >= 256 k per split
   if (max_split > 16) max_split = 16;

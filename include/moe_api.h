@@ -41,7 +41,9 @@
  *    moe_read_device_error.
  *  - Limits: 1 <= top_k <= min(E, 32), E <= 1024, d and ffn multiples of 8,
  *    T*top_k < 2^31. Outside them a call returns MOE_ERR_UNSUPPORTED (or
- *    MOE_ERR_INVALID_ARG for nonsensical values). T == 0 is a no-op.
+ *    MOE_ERR_INVALID_ARG for nonsensical values). T == 0 is a no-op: once
+ *    the config passes its checks the call returns MOE_OK without looking
+ *    at any pointer (empty buffers may be null) and launches nothing.
  *  - Workspace: every call that takes `ws` needs ws_bytes >=
  *    moe_workspace_size(cfg) and a 256-byte aligned `ws`; the same workspace
  *    serves all calls of one config. Its first 256 bytes hold the device

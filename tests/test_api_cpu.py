@@ -46,6 +46,8 @@ def test_workspace_size_valid_and_invalid(L):
     nb = L.moe_workspace_size(ctypes.byref(big))
     # holds at least x_perm, h and y_perm for T*k rows
     assert nb >= 16384 * 8 * (4096 * 2 + 1024) * 2
+    # an empty batch has a (small) workspace too
+    assert 0 < L.moe_workspace_size(ctypes.byref(cfg(T=0))) < n
     for bad in (cfg(k=0), cfg(k=11), cfg(d=0), cfg(T=-1), cfg(N=0, Z=0),
                 cfg(dt=7), cfg(k=33, N=40), cfg(N=1020, Z=10), cfg(d=260),
                 cfg(F=100), cfg(s=float("inf"))):
@@ -126,6 +128,23 @@ def test_pointer_errors_before_launch(L):
     assert L.moe_layer_forward_host(ctypes.byref(c), None, *ok[1:6], ok[6], None,
                                     ok[8], ws_n, st) == 1
     assert L.moe_read_device_error(None, None, st) == 3
+
+
+def test_empty_batch_is_a_no_op_before_any_pointer_check(L):
+    # T == 0: every entry point returns MOE_OK with all pointers null (empty
+    # buffers have no address) and no workspace; nothing is launched, so this
+    # runs without a GPU. A bad config is still an error.
+    c = cfg(T=0)
+    st = P(0)
+    assert L.moe_route(ctypes.byref(c), *[None] * 8, 0, st) == 0
+    assert L.moe_route_noalloc(ctypes.byref(c), *[None] * 7, st) == 0
+    assert L.moe_dispatch(ctypes.byref(c), *[None] * 8, 0, st) == 0
+    assert L.moe_expert_ffn(ctypes.byref(c), *[None] * 7, 0, st) == 0
+    assert L.moe_combine(ctypes.byref(c), *[None] * 6, st) == 0
+    assert L.moe_layer_forward(ctypes.byref(c), *[None] * 9, 0, st) == 0
+    assert L.moe_layer_forward_host(ctypes.byref(c), *[None] * 9, 0, st) == 0
+    bad = cfg(T=0, k=11)
+    assert L.moe_layer_forward(ctypes.byref(bad), *[None] * 9, 0, st) == 1
 
 
 def test_python_binding_marshalling_checks():

@@ -1,5 +1,5 @@
 """GPU edge cases of the layer, each against the oracle or an exact property:
-T = 1, every slot on zero experts (R = 0: the expert GEMMs launch no work),
+T = 0 and T = 1, every slot on zero experts (R = 0: the expert GEMMs launch no work),
 every token on one expert, segment sizes around the 128-row token tile,
 only zero experts (N = 0), no zero experts (Z = 0), k = E, the largest
 supported E and k, and the device-side wait limit (a wait that nothing
@@ -199,6 +199,28 @@ def test_router_exact_ties_go_to_lower_id():
     np.testing.assert_array_equal(idx.cpu().numpy(), ref_idx)
     np.testing.assert_array_equal(ref_idx, np.tile(np.arange(3, 9), (sh.T, 1)))
     np.testing.assert_allclose(gate.cpu().numpy(), 1.0 / 6, rtol=1e-6)
+
+
+def test_empty_batch():
+    # T = 0 through every binding call: empty outputs, no launch, no device
+    # error; the same workspace then serves a real batch of the same layer
+    sh = MoEShape("empty", T=0, d=256, n_routed=8, n_zero=2, top_k=2, ffn=256)
+    inp = make_inputs(sh, 15)
+    ls = shape_of(sh)
+    d = inp.to(DEV)
+    ws = moe.alloc_workspace(ls)
+    idx, gate = moe.route(ls, d.x, d.w_router, d.bias, ws)
+    assert idx.shape == (0, 2) and gate.shape == (0, 2)
+    counts, offsets, row_token, slot_row, x_perm = moe.dispatch(ls, d.x, idx, ws)
+    y = moe.expert_ffn(ls, x_perm, offsets, d.w_gate, d.w_up, d.w_down, ws)
+    out = moe.combine(ls, d.x, y, idx, gate, slot_row)
+    assert out.shape == (0, sh.d)
+    out = moe.layer_forward(ls, d.x, d.w_router, d.bias, d.w_gate, d.w_up, d.w_down, ws)
+    assert out.shape == (0, sh.d)
+    torch.cuda.synchronize()
+    assert moe.read_device_error(ws) == 0
+    full = MoEShape("after_empty", T=24, d=256, n_routed=8, n_zero=2, top_k=2, ffn=256)
+    check_layer(full, make_inputs(full, 16))
 
 
 def test_wait_limit_reports_and_context_stays_usable():
