@@ -638,6 +638,7 @@ int64_t router_planes_rows(const Shape& sh) { return (3 * sh.E + 127) / 128 * 12
 // elements (16 blocks of 64), a chain of 64 MMA steps per partial.
 static int router_kb_chunk(const Shape& sh) {
   const int kb = (int)(sh.d / 64);
+  if (kb < 1) return 1;  // d < 64: the tensor-core router is not used, but sizes stay defined
   int c = kb < 16 ? kb : 16;
   while (kb % c != 0) --c;
   return c;

@@ -55,6 +55,19 @@ def test_workspace_size_valid_and_invalid(L):
     assert L.moe_workspace_size(None) == 0
 
 
+def test_host_sizing_defined_across_the_limits(L):
+    # workspace size and launch count for every d the limits allow up to 1024,
+    # at batch sizes on both sides of each path threshold: each is defined
+    # (no division by an empty count) and the config is accepted
+    for d in range(8, 1025, 8):
+        for T in (0, 1, 63, 257, 512, 1025, 4097):
+            for dt in (moe.MOE_BF16, moe.MOE_F32):
+                for N, Z, k, F in ((6, 2, 2, 8), (1, 0, 1, 256), (0, 3, 2, 128)):
+                    c = cfg(T=T, d=d, N=N, Z=Z, k=k, F=F, dt=dt)
+                    assert L.moe_workspace_size(ctypes.byref(c)) > 0, (d, T, dt, N, F)
+                    assert L.moe_layer_launch_count(ctypes.byref(c)) >= 0
+
+
 def test_launch_count(L):
     # router 1 (T <= 256), 2 (CUDA cores) or 3 (split + tensor-core GEMM +
     # top-k); dispatch 1 (one block for T <= 4096) or 3, + gather unless the
