@@ -8,7 +8,9 @@ Paths covered (by the rules the host applies): the one-launch small router
 router (bf16, T >= 512); the one-block and multi-kernel dispatch; the
 CUDA-core FFN (f32, or d or F not a multiple of 128); single-CTA tensor-core
 GEMMs with 64-, 128- and 256-token tiles, with and without a split
-contraction; and the CTA-pair GEMMs with their dynamic schedule.
+contraction; and the CTA-pair GEMMs with their dynamic schedule. Also the
+narrowest widths the limits allow, a single routed expert (a dense FFN), and
+one token past each batch-size threshold.
 """
 import pytest
 
@@ -42,6 +44,20 @@ SHAPES = [
     MoEShape("fz_t90_simt", T=90, d=200, n_routed=6, n_zero=2, top_k=2, ffn=136),
     MoEShape("fz_t50_f32", T=50, d=128, n_routed=5, n_zero=1, top_k=3, ffn=128,
              act_dtype="f32"),
+    # the narrowest layers the limits allow (router boxes wider than the rows)
+    MoEShape("fz_d8", T=33, d=8, n_routed=3, n_zero=1, top_k=2, ffn=8),
+    MoEShape("fz_d16_f32", T=20, d=16, n_routed=4, n_zero=2, top_k=3, ffn=24,
+             act_dtype="f32"),
+    # one routed expert: a dense SwiGLU FFN on tensor cores, with and without
+    # zero experts beside it
+    MoEShape("fz_dense", T=100, d=256, n_routed=1, n_zero=0, top_k=1, ffn=256),
+    MoEShape("fz_n1_zero", T=70, d=128, n_routed=1, n_zero=3, top_k=2, ffn=128),
+    # one token past each batch-size threshold: small router (256), tensor-core
+    # router (512), CTA pairs (1024), one-block dispatch (4096)
+    MoEShape("fz_t257", T=257, d=128, n_routed=6, n_zero=2, top_k=2, ffn=128),
+    MoEShape("fz_t512", T=512, d=128, n_routed=6, n_zero=2, top_k=2, ffn=128),
+    MoEShape("fz_t1025_pairs", T=1025, d=256, n_routed=4, n_zero=1, top_k=1, ffn=256),
+    MoEShape("fz_t4097", T=4097, d=128, n_routed=8, n_zero=2, top_k=2, ffn=128),
 ]
 
 
