@@ -145,9 +145,11 @@ def run_reference(args, sh):
     if rank != 0:
         return
     inp = make_inputs(sh, args.seed)
-    sample = min(sh.T, args.ref_tokens)
-    toks = torch.arange(sample, dtype=torch.int32).numpy()
     cores = oracle.num_threads()
+    # the oracle runs its tokens in parallel, one per thread: by default a
+    # step samples one token per host thread, so every core has work
+    sample = min(sh.T, args.ref_tokens if args.ref_tokens else cores)
+    toks = torch.arange(sample, dtype=torch.int32).numpy()
 
     def step():
         oracle.layer(inp.x, inp.w_router, inp.bias, inp.w_gate, inp.w_up, inp.w_down,
@@ -481,7 +483,8 @@ def main():
     ap.add_argument("--config", default="decode")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--ref-tokens", type=int, default=8)
+    ap.add_argument("--ref-tokens", type=int, default=0,
+                    help="tokens per reference step (default: one per host thread)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
