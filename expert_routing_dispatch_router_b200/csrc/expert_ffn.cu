@@ -929,16 +929,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
+  // looked up once; callers on several host threads may race to store the
+  // same pointer, hence the atomic
+  static std::atomic<PFN_cuTensorMapEncodeTiled_v12000> fn{nullptr};
+  if (!fn.load()) {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
             cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+      fn.store(reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p));
   }
-  return fn;
+  return fn.load();
 }
 
 // Row-major bf16 matrix [rows, cols] seen as a 2-D tensor, box = 64 columns
