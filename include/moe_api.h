@@ -36,9 +36,9 @@
  *    rows, because the number R of routed rows is only known on the device.
  *  - Errors: argument errors are found on the host before anything is
  *    launched and leave every buffer untouched. A launch failure returns
- *    MOE_ERR_CUDA. Device-side checks (a bounded wait in the expert GEMM that
- *    ran out) are recorded in the workspace and reported by
- *    moe_read_device_error.
+ *    MOE_ERR_CUDA. Device-side checks (a bounded wait in the router or an
+ *    expert GEMM that ran out; an invalid expert id given to the dispatch)
+ *    are recorded in the workspace and reported by moe_read_device_error.
  *  - Limits: 1 <= top_k <= min(E, 32), E <= 1024, d and ffn multiples of 8,
  *    T*top_k < 2^31. Outside them a call returns MOE_ERR_UNSUPPORTED (or
  *    MOE_ERR_INVALID_ARG for nonsensical values). T == 0 is a no-op: once
@@ -222,11 +222,12 @@ moe_status_t moe_bias_pid_update(const moe_config_t* cfg, const int32_t* counts,
                                  const moe_pid_params_t* params, moe_stream_t stream);
 
 /* Waits for `stream`, then reads and clears the device-side error word in ws.
- * *code_out (may be NULL) gets 0 when no check failed, else a nonzero code
- * (1 = a bounded wait in the router or an expert GEMM ran out, 2 = a routing slot held an
- * expert id outside [0, E) or one token listed an expert twice; such slots
- * are skipped). Returns
- * MOE_ERR_DEVICE_CHECK when the code is nonzero. */
+ * *code_out (may be NULL) gets 0 when no check failed, else a nonzero code:
+ *   1 = a bounded wait in the router or an expert GEMM ran out (2 s);
+ *   2 = a routing slot held an expert id outside [0, E), or one token listed
+ *       an expert twice; such slots are skipped.
+ * Returns MOE_ERR_DEVICE_CHECK when the code is nonzero, MOE_ERR_WORKSPACE
+ * for a NULL ws. */
 moe_status_t moe_read_device_error(void* ws, int32_t* code_out,
                                    moe_stream_t stream);
 
