@@ -27,7 +27,7 @@
  *    "底层定制算子深度优化": Dispatch/Combine operators that support
  *    zero-computation experts.
  *
- * Readings where the pages are silent (each is listed in the design notes):
+ * Readings taken where the pages are silent or ambiguous:
  *  R1 expert ids 0..N-1 are routed, N..E-1 are zero experts;
  *  R2 the correction bias is added to the logits for selection only;
  *  R3 the selected set is the k largest keys, ties to the lower id, emitted in
@@ -353,10 +353,11 @@ void oracle_layer(int64_t n_tok, const int32_t* tokens, int64_t T, int64_t d,
 
 /* ------------------------------------------------- router bias controller -- */
 
-/* PID update of the zero experts' router bias, reading R13 (see the design
- * notes): "Meituan lancerer LongCat-2.0" (snilld.dk), "MoE i praksis og
- * prisen for fleksibilitet", says a PID controller adjusts the router bias so
- * that the activation stays in the wanted range. The controlled value is the
+/* PID update of the zero experts' router bias (reading R13). "Meituan
+ * lancerer LongCat-2.0" (snilld.dk), "MoE i praksis og prisen for
+ * fleksibilitet", says a PID controller adjusts the router bias so that the
+ * activation stays in the wanted range, and gives no gains, set-point or
+ * controlled variable. Here the controlled value is the
  * share of routing slots that went to routed experts,
  *   share = sum_{e<N} counts[e] / (T k),
  * the error is err = share - target, and
