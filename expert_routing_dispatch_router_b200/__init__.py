@@ -131,13 +131,28 @@ def _check(fn: str, status: int):
         raise MoEError(fn, status, lib().moe_status_string(status).decode())
 
 
-def _need(t: torch.Tensor, name: str, dtype, shape=None):
+def _need(t: torch.Tensor, name: str, dtype, shape=None, on_device=True):
+    """Checks one tensor argument before its address goes to the library. A
+    host tensor where device memory is expected (or the reverse) would be
+    dereferenced by a kernel or a copy on the wrong side, so it is refused."""
     if t.dtype != dtype:
         raise ValueError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if on_device and not t.is_cuda:
+        raise ValueError(f"{name}: must be a CUDA tensor")
+    if not on_device and t.is_cuda:
+        raise ValueError(f"{name}: must be a host tensor")
     if not t.is_contiguous():
         raise ValueError(f"{name}: must be contiguous")
     if shape is not None and tuple(t.shape) != tuple(shape):
         raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _ws(ws: torch.Tensor):
+    """(address, size in bytes) of a workspace tensor, which must be device
+    memory (alloc_workspace gives one)."""
+    if not ws.is_cuda or not ws.is_contiguous():
+        raise ValueError("ws: must be a contiguous CUDA tensor (use alloc_workspace)")
+    return ctypes.c_void_p(ws.data_ptr()), ws.numel() * ws.element_size()
 
 
 def workspace_size(shape: LayerShape) -> int:
@@ -170,8 +185,8 @@ def route(shape: LayerShape, x, w_router, bias, ws, logits=None, flags=None,
     if flags is not None:
         _need(flags, "flags", torch.uint8, (T,))
     st = lib().moe_route(ctypes.byref(shape.c()), _ptr(x), _ptr(w_router), _ptr(bias),
-                         _ptr(logits), _ptr(idx), _ptr(gate), _ptr(flags), _ptr(ws),
-                         ws.numel(), _stream(stream))
+                         _ptr(logits), _ptr(idx), _ptr(gate), _ptr(flags), *_ws(ws),
+                         _stream(stream))
     _check("moe_route", st)
     return idx, gate
 
@@ -212,7 +227,7 @@ def dispatch(shape: LayerShape, x, topk_idx, ws, stream=None):
     x_perm = torch.empty(T * k, shape.d, dtype=shape.act_dtype, device=dev)
     st = lib().moe_dispatch(ctypes.byref(shape.c()), _ptr(x), _ptr(topk_idx),
                             _ptr(counts), _ptr(offsets), _ptr(row_token),
-                            _ptr(slot_row), _ptr(x_perm), _ptr(ws), ws.numel(),
+                            _ptr(slot_row), _ptr(x_perm), *_ws(ws),
                             _stream(stream))
     _check("moe_dispatch", st)
     return counts, offsets, row_token, slot_row, x_perm
@@ -232,7 +247,7 @@ def expert_ffn(shape: LayerShape, x_perm, offsets, w_gate, w_up, w_down, ws,
     _need(y_perm, "y_perm", torch.float32, (T * k, d))
     st = lib().moe_expert_ffn(ctypes.byref(shape.c()), _ptr(x_perm), _ptr(offsets),
                               _ptr(w_gate), _ptr(w_up), _ptr(w_down), _ptr(y_perm),
-                              _ptr(ws), ws.numel(), _stream(stream))
+                              *_ws(ws), _stream(stream))
     _check("moe_expert_ffn", st)
     return y_perm
 
@@ -273,7 +288,7 @@ def layer_forward(shape: LayerShape, x, w_router, bias, w_gate, w_up, w_down, ws
         _need(counts, "counts", torch.int32, (E,))
     st = lib().moe_layer_forward(ctypes.byref(shape.c()), _ptr(x), _ptr(w_router),
                                  _ptr(bias), _ptr(w_gate), _ptr(w_up), _ptr(w_down),
-                                 _ptr(out), _ptr(counts), _ptr(ws), ws.numel(),
+                                 _ptr(out), _ptr(counts), *_ws(ws),
                                  _stream(stream))
     _check("moe_layer_forward", st)
     return out
@@ -284,16 +299,21 @@ def layer_forward_host(shape: LayerShape, x_host, w_router, bias, w_gate, w_up,
     """The whole layer with x and out in (pinned) host memory; asynchronous:
     synchronise the stream before reading out_host."""
     T, d, E = shape.T, shape.d, shape.E
-    _need(x_host, "x_host", shape.act_dtype, (T, d))
-    _need(out_host, "out_host", shape.act_dtype, (T, d))
-    if x_host.is_cuda or out_host.is_cuda:
-        raise ValueError("x_host and out_host must be host tensors")
+    F, N = shape.ffn, shape.n_routed
+    _need(x_host, "x_host", shape.act_dtype, (T, d), on_device=False)
+    _need(out_host, "out_host", shape.act_dtype, (T, d), on_device=False)
     if counts_host is not None:
-        _need(counts_host, "counts_host", torch.int32, (E,))
+        _need(counts_host, "counts_host", torch.int32, (E,), on_device=False)
+    _need(w_router, "w_router", torch.float32, (E, d))
+    _need(bias, "bias", torch.float32, (E,))
+    if N > 0:
+        for name, w, shp in (("w_gate", w_gate, (N, F, d)), ("w_up", w_up, (N, F, d)),
+                             ("w_down", w_down, (N, d, F))):
+            _need(w, name, shape.act_dtype, shp)
     st = lib().moe_layer_forward_host(ctypes.byref(shape.c()), _ptr(x_host),
                                       _ptr(w_router), _ptr(bias), _ptr(w_gate),
                                       _ptr(w_up), _ptr(w_down), _ptr(out_host),
-                                      _ptr(counts_host), _ptr(ws), ws.numel(),
+                                      _ptr(counts_host), *_ws(ws),
                                       _stream(stream))
     _check("moe_layer_forward_host", st)
     return out_host
@@ -302,7 +322,7 @@ def layer_forward_host(shape: LayerShape, x_host, w_router, bias, w_gate, w_up,
 def read_device_error(ws, stream=None) -> int:
     """Waits for the stream; returns (and clears) the workspace error word."""
     code = ctypes.c_int32(0)
-    lib().moe_read_device_error(_ptr(ws), ctypes.byref(code), _stream(stream))
+    lib().moe_read_device_error(_ws(ws)[0], ctypes.byref(code), _stream(stream))
     return int(code.value)
 
 
@@ -310,7 +330,7 @@ def selftest_wait_limit(ws, stream=None) -> None:
     """Runs the device-side wait-limit self-test: after ~2 s the workspace
     error word holds 1 (read it with read_device_error)."""
     _check("moe_selftest_wait_limit",
-           lib().moe_selftest_wait_limit(_ptr(ws), ws.numel() * ws.element_size(),
+           lib().moe_selftest_wait_limit(*_ws(ws),
                                          _stream(stream)))
 
 

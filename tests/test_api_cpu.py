@@ -160,6 +160,27 @@ def test_empty_batch_is_a_no_op_before_any_pointer_check(L):
     assert L.moe_layer_forward(ctypes.byref(bad), *[None] * 9, 0, st) == 1
 
 
+def test_binding_refuses_host_tensors_for_device_arguments():
+    # a host tensor's address handed to a kernel would fault the GPU: the
+    # binding refuses it before the library is called (runs without a GPU)
+    import torch
+    sh = moe.LayerShape(T=4, d=64, n_routed=2, n_zero=1, top_k=2, ffn=64)
+    x = torch.zeros(4, 64, dtype=torch.bfloat16)
+    w_r, b = torch.zeros(3, 64), torch.zeros(3)
+    wg, wd = torch.zeros(2, 64, 64, dtype=torch.bfloat16), torch.zeros(2, 64, 64,
+                                                                        dtype=torch.bfloat16)
+    ws = torch.zeros(1 << 20, dtype=torch.uint8)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        moe.layer_forward(sh, x, w_r, b, wg, wg, wd, ws)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        moe.route(sh, x, w_r, b, ws)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        moe.read_device_error(ws)
+    # the host entry point checks its device weights as well as its host buffers
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        moe.layer_forward_host(sh, x, w_r, b, wg, wg, wd, ws, torch.zeros_like(x))
+
+
 def test_python_binding_marshalling_checks():
     import torch
     sh = moe.LayerShape(T=4, d=64, n_routed=2, n_zero=1, top_k=2, ffn=64)
