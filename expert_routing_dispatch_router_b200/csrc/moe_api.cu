@@ -87,6 +87,7 @@ moe_status_t make_shape(const moe_config_t* c, Shape* sh) {
   sh->es = sh->bf16 ? 2 : 4;
   sh->s = c->routed_scale;
   sh->nchunks = (sh->T + kChunkTokens - 1) / kChunkTokens;
+  if (!router_grid_fits(*sh)) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
 

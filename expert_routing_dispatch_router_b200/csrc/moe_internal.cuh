@@ -109,6 +109,9 @@ bool router_uses_tensor_cores(const Shape& sh);
 int64_t router_planes_rows(const Shape& sh);   // 3E rounded up to 128
 int router_tc_chunks(const Shape& sh);         // contraction chunks of that router
 int router_launch_count(const Shape& sh);
+// False when the batch is too large for the router path it would take (the
+// CUDA-core router tiles tokens along gridDim.y, at most 65535 tiles).
+bool router_grid_fits(const Shape& sh);
 int router_small_splits(const Shape& sh);
 int expert_ffn_launch_count(const Shape& sh);
 cudaError_t launch_bias_pid(const Shape& sh, const int32_t* counts, float* bias,

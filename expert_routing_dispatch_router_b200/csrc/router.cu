@@ -683,6 +683,11 @@ int router_small_plan(const Shape& sh, int* ksplit_out) {
 
 int router_small_splits(const Shape& sh) { return router_small_plan(sh, nullptr); }
 
+bool router_grid_fits(const Shape& sh) {
+  if (router_uses_tensor_cores(sh) || router_uses_small_kernel(sh)) return true;
+  return (sh.T + RT - 1) / RT <= 65535;
+}
+
 int router_launch_count(const Shape& sh) {
   return router_uses_tensor_cores(sh) ? 3 : (router_uses_small_kernel(sh) ? 1 : 2);
 }

@@ -40,7 +40,8 @@
  *    expert GEMM that ran out; an invalid expert id given to the dispatch)
  *    are recorded in the workspace and reported by moe_read_device_error.
  *  - Limits: 1 <= top_k <= min(E, 32), E <= 1024, d and ffn multiples of 8,
- *    T*top_k < 2^31. Outside them a call returns MOE_ERR_UNSUPPORTED (or
+ *    T*top_k < 2^31, and T <= 4194240 where the router runs on CUDA cores
+ *    (f32 activations above 256 tokens, or d not a multiple of 128). Outside them a call returns MOE_ERR_UNSUPPORTED (or
  *    MOE_ERR_INVALID_ARG for nonsensical values). T == 0 is a no-op: once
  *    the config passes its checks the call returns MOE_OK without looking
  *    at any pointer (empty buffers may be null) and launches nothing.

@@ -68,6 +68,19 @@ def test_host_sizing_defined_across_the_limits(L):
                     assert L.moe_layer_launch_count(ctypes.byref(c)) >= 0
 
 
+def test_cuda_core_router_token_limit(L):
+    # the CUDA-core router (f32, or d not a multiple of 128) takes at most
+    # 65535 tiles of 64 tokens; beyond that the config is refused up front
+    for dt, d in ((moe.MOE_F32, 128), (moe.MOE_BF16, 64)):
+        ok = cfg(T=65535 * 64, d=d, N=2, Z=1, k=1, F=8, dt=dt)
+        over = cfg(T=65535 * 64 + 1, d=d, N=2, Z=1, k=1, F=8, dt=dt)
+        assert L.moe_workspace_size(ctypes.byref(ok)) > 0
+        assert L.moe_workspace_size(ctypes.byref(over)) == 0
+    # the tensor-core router (bf16, d a multiple of 128) has no such limit
+    big = cfg(T=65535 * 64 + 1, d=128, N=2, Z=1, k=1, F=8)
+    assert L.moe_workspace_size(ctypes.byref(big)) > 0
+
+
 def test_launch_count(L):
     # router 1 (T <= 256), 2 (CUDA cores) or 3 (split + tensor-core GEMM +
     # top-k); dispatch 1 (one block for T <= 4096) or 3, + gather unless the
