@@ -44,10 +44,13 @@ def build(force: bool = False) -> str:
 
 
 def _load():
+    """The compiled oracle. MOE_ORACLE_LIB, when set, names a compiled variant
+    of moe_oracle.c to load instead: the test that plants mistakes in the
+    oracle uses it to check that the pins catch each one."""
     global _lib
     with _lock:
         if _lib is None:
-            lib = ctypes.CDLL(build())
+            lib = ctypes.CDLL(os.environ.get("MOE_ORACLE_LIB") or build())
             P, I64, I, D = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_double
             sig = {
                 "oracle_num_threads": ([], I),
