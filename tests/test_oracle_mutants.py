@@ -13,7 +13,8 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "moe_oracle.c")
 PINS = [os.path.join(ROOT, "tests", "test_oracle_pins.py"),
-        os.path.join(ROOT, "tests", "test_oracle_bruteforce.py")]
+        os.path.join(ROOT, "tests", "test_oracle_bruteforce.py"),
+        os.path.join(ROOT, "tests", "test_bias_pid.py")]
 
 # (name, text in the source, replacement, occurrences); every planted mistake
 # keeps all accesses in bounds
@@ -42,6 +43,10 @@ MUTANTS = [
      "for (int64_t t = T - 1; t >= 0; --t)\n      for (int64_t j = 0; j < k; ++j)\n        if (idx[t * k + j] == e) {",
      1),
     ("margin_sign", "*margin = kth_key - next;", "*margin = next - kth_key;", 1),
+    ("pid_integral_not_carried", "const double integral = state[0] + err;",
+     "const double integral = err;", 1),
+    ("pid_derivative_sign", "kd * (err - state[1]);", "kd * (state[1] - err);", 1),
+    ("pid_no_clamp", "if (u > max_step) u = max_step;", "(void)max_step;", 1),
 ]
 
 
@@ -58,8 +63,8 @@ def _compile(text, directory, name):
 def _run_pins(lib):
     env = dict(os.environ, MOE_ORACLE_LIB=lib, OMP_NUM_THREADS="2")
     return subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
-                           *PINS], cwd=ROOT, env=env, capture_output=True, text=True,
-                          timeout=900)
+                           "-m", "not gpu", *PINS], cwd=ROOT, env=env, capture_output=True,
+                          text=True, timeout=900)
 
 
 @pytest.fixture(scope="module")
