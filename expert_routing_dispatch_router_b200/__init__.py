@@ -7,6 +7,11 @@ tensors into that ABI (pointers, sizes, the current stream); it computes
 nothing itself and has no fallback: if the library is missing, importing the
 binding's functions raises.
 
+All CUDA tensors of a call must live on the current device
+(``torch.cuda.set_device``): the library launches its kernels there, on the
+given stream or that device's current stream, and they read the tensors
+directly.
+
 Build the library with ``python -m expert_routing_dispatch_router_b200.build``.
 """
 from __future__ import annotations

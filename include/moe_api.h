@@ -24,7 +24,9 @@
  *    synchronises nothing (moe_read_device_error is the one call that waits,
  *    and only on the stream it is given).
  *  - Pointers are device pointers unless the name ends in _host. All tensors
- *    are dense row-major. Every pointer must be 16-byte aligned.
+ *    are dense row-major. Every pointer must be 16-byte aligned. The device
+ *    pointers of a call must all be memory of the current CUDA device, the
+ *    one `stream` belongs to: kernels run there and read them directly.
  *  - act_dtype is the type of x, out, the expert weights and x_perm:
  *    MOE_F32 (float) or MOE_BF16 (bfloat16). w_router, bias, topk_gate and
  *    the expert outputs y_perm are always float; indices are int32. (y_perm
