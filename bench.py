@@ -5,8 +5,11 @@
 
 One step = one pass of the whole layer (router + top-k, dispatch, grouped
 SwiGLU expert GEMMs, combine) over one batch of seeded synthetic tokens. The
-default workload is the bf16 decode layer (T=64, d=4096, 128 routed experts of
-width 1024 + 32 zero experts, top-8, fp32 router). Prints one JSON line.
+default workload is the largest fixed single-GPU layer, the bf16
+large-expert-count layer (T=8192, d=6144, 256 routed experts of width 2048 +
+64 zero experts, top-12, fp32 router, about 30 % of routing slots on zero
+experts); ``--config decode`` and the others select the remaining workloads.
+Prints one JSON line.
 
 Under torchrun each rank runs its own replica on its own batch (seed + rank):
 the layer is data-parallel over tokens with no exchange, so scaling is weak
@@ -79,6 +82,15 @@ def workload_name(sh):
     return (f"{sh.name}: T={sh.T}, d={sh.d}, {sh.n_routed} routed experts (SwiGLU, "
             f"F={sh.ffn}) + {sh.n_zero} zero experts, top-{sh.top_k}, "
             f"{sh.act_dtype} activations/weights, fp32 router, routing={sh.routing}")
+
+
+def run_config(sh, seed, world):
+    """The `config` object of the JSON line; both arms print the same one."""
+    w_bytes = sh.n_routed * 3 * sh.ffn * sh.d * (2 if sh.act_dtype == "bf16" else 4)
+    return {"workload": workload_name(sh), "seed": seed,
+            "l2": "inputs larger than L2: the touched expert weights (up to "
+                  f"{w_bytes / 1e9:.2f} GB) stream from HBM every step",
+            "parallelism": f"replicas{world}"}
 
 
 # ------------------------------------------------------------------ clocks --
@@ -167,7 +179,7 @@ def run_reference(args, sh):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": workload_name(sh), "seed": args.seed},
+        "config": run_config(sh, args.seed, int(os.environ.get("WORLD_SIZE", "1"))),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores,
                          "kind": "oracle",
                          "sample": f"per step: whole layer on the first {sample} of "
@@ -453,12 +465,9 @@ def run_gpu(args, sh):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": sh.act_dtype, "data": "synthetic",
-            "config": {"workload": workload_name(sh), "seed": args.seed,
-                       "l2": "inputs larger than L2: the touched expert weights "
-                             f"({U} experts, {U * 3 * sh.ffn * sh.d * 2 / 1e9:.2f} GB) "
-                             "stream from HBM every step",
-                       "parallelism": f"replicas{world}",
-                       "launch": f"CUDA graph of {G} layer calls, replayed {args.steps // G} times"},
+            "config": run_config(sh, args.seed, world),
+            "launch": f"CUDA graph of {G} layer calls, replayed {args.steps // G} times",
+            "touched_experts": {"U": U, "weight_bytes": U * 3 * sh.ffn * sh.d * 2},
             "e2e": {"value": replicas.job_throughput(sh.T, 1, info, e2e_ms[2]), "unit": "tokens/s",
                     "launch": f"CUDA graph of {G} host-entry calls alternating between two "
                               "streams and workspaces (copies included)",
@@ -480,7 +489,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--config", default="decode")
+    ap.add_argument("--config", default="large_e")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-tokens", type=int, default=0,

@@ -12,7 +12,9 @@
 // which every GPU that loads this library holds until the process exits. The
 // first call on a device, with that device current, looks up the array's
 // device address once (cudaGetSymbolAddress) and remembers it; make that first
-// call before any stream capture on the device. Every call on a device shares
+// call before any stream capture on the device. The remembered address belongs
+// to the device's primary context: after cudaDeviceReset on that device the
+// process must not call this entry point again. Every call on a device shares
 // the one array and leaves the last call's partial sums in it. Nothing has to
 // start at zero: each call writes every partial sum it later reads. Calls
 // whose work overlaps on the GPU (other streams, other host threads) race on
@@ -27,6 +29,7 @@ cudaError_t launch_router_simt(const Shape& sh, const void* x, const float* w_r,
                                int32_t* idx, float* gate, uint8_t* flags,
                                float* logits_out, cudaStream_t st);
 int router_splits(const Shape& sh);
+bool router_simt_grid_fits(const Shape& sh);
 moe_status_t shape_from_config(const moe_config_t* c, Shape* sh);
 }  // namespace moe
 
@@ -76,9 +79,14 @@ extern "C" moe_status_t moe_route_noalloc(const moe_config_t* cfg, const void* x
       !aligned16(topk_idx) || !aligned16(topk_gate) || !aligned16(logits) ||
       !aligned16(flags))
     return MOE_ERR_INVALID_ARG;
-  // the partial sums of one split need T * E floats
+  // this call always runs the CUDA-core router, whatever path moe_route would
+  // take for the shape, so its grid limit is checked here too; the partial
+  // sums of one split need T * E floats
   const int64_t per_split = sh.T * sh.E;
-  if (per_split > kNoAllocScratchFloats) return MOE_ERR_UNSUPPORTED;
+  if (per_split > kNoAllocScratchFloats || !router_simt_grid_fits(sh))
+    return MOE_ERR_UNSUPPORTED;
+  // router_splits keeps nsplit * T * E near 2 * SMs * RT * RE (~0.6 M floats),
+  // so this clamp only guards the array against a future split rule
   int nsplit = router_splits(sh);
   if ((int64_t)nsplit * per_split > kNoAllocScratchFloats)
     nsplit = (int)(kNoAllocScratchFloats / per_split);

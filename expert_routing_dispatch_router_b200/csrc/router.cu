@@ -683,9 +683,12 @@ int router_small_plan(const Shape& sh, int* ksplit_out) {
 
 int router_small_splits(const Shape& sh) { return router_small_plan(sh, nullptr); }
 
+// The CUDA-core logits GEMM puts token tiles of RT on grid.y (at most 65535).
+bool router_simt_grid_fits(const Shape& sh) { return (sh.T + RT - 1) / RT <= 65535; }
+
 bool router_grid_fits(const Shape& sh) {
   if (router_uses_tensor_cores(sh) || router_uses_small_kernel(sh)) return true;
-  return (sh.T + RT - 1) / RT <= 65535;
+  return router_simt_grid_fits(sh);
 }
 
 int router_launch_count(const Shape& sh) {

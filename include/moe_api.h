@@ -185,10 +185,13 @@ moe_status_t moe_layer_forward_host(const moe_config_t* cfg, const void* x_host,
  *  always runs the CUDA-core router). It allocates nothing: its scratch is
  *  one 16 MiB array inside the library, held by every GPU that loads the
  *  library until the process exits.
- *  Limit: T * (n_routed + n_zero) <= 4194304; larger problems return
- *  MOE_ERR_UNSUPPORTED before anything is launched.
+ *  Limits: T * (n_routed + n_zero) <= 4194304, and T <= 65535 * 64 (the
+ *  CUDA-core router's grid); larger problems return MOE_ERR_UNSUPPORTED
+ *  before anything is launched.
  *  The first call on a device (with that device current) looks up the
  *  array's address once; make it before any stream capture on that device.
+ *  The address is kept for the life of the process: after cudaDeviceReset
+ *  on a device, do not call this entry point on it again.
  *  All calls on a device share the array: calls that overlap on the GPU
  *  (other streams or host threads) race and must be ordered by the caller. */
 moe_status_t moe_route_noalloc(const moe_config_t* cfg, const void* x,

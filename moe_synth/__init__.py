@@ -92,6 +92,11 @@ CONFIGS: Dict[str, MoEShape] = {
     # the large-expert layer's density (~270 rows per expert), 32 experts
     "profile_large_e": MoEShape("profile_large_e", T=1024, d=6144, n_routed=32,
                                 n_zero=8, top_k=12, ffn=2048),
+    # the same density above 1024 tokens, where the expert GEMMs run on CTA
+    # pairs: 64 routed + 28 zero experts (~70 % routed slots, ~270 rows per
+    # expert), 4.8 GB of weights
+    "profile_large_e_pairs": MoEShape("profile_large_e_pairs", T=2048, d=6144,
+                                      n_routed=64, n_zero=28, top_k=12, ffn=2048),
 }
 
 SWEEP_T = (1, 8, 64, 512, 4096, 32768)

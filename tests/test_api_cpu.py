@@ -156,6 +156,23 @@ def test_pointer_errors_before_launch(L):
     assert L.moe_read_device_error(None, None, st) == 3
 
 
+def test_route_noalloc_refuses_problems_beyond_its_limits(L):
+    # moe_route_noalloc checks its limits on the host before it looks up its
+    # scratch array or launches anything, so fake device addresses never reach
+    # a kernel (runs without a GPU)
+    st = P(0)
+    # T * E beyond the 16 MiB scratch array
+    c = cfg(T=32768, d=256, N=121, Z=8, k=4, F=128)
+    assert L.moe_route_noalloc(ctypes.byref(c), _fake(), _fake(), _fake(), None, _fake(),
+                               _fake(), None, st) == 2
+    # T * E within the array, but more token tiles than the CUDA-core router's
+    # grid takes (moe_route would run this shape on the tensor cores)
+    c = cfg(T=65536 * 64, d=128, N=1, Z=0, k=1, F=8)
+    assert L.moe_workspace_size(ctypes.byref(c)) > 0
+    assert L.moe_route_noalloc(ctypes.byref(c), _fake(), _fake(), _fake(), None, _fake(),
+                               _fake(), None, st) == 2
+
+
 def test_empty_batch_is_a_no_op_before_any_pointer_check(L):
     # T == 0: every entry point returns MOE_OK with all pointers null (empty
     # buffers have no address) and no workspace; nothing is launched, so this

@@ -34,6 +34,20 @@ def test_reference_line_has_the_contract_keys():
     # one sampled token per oracle thread (at most T)
     assert f"first {min(128, j['cpu_baseline']['cores'])} of 128 tokens" in \
         j["cpu_baseline"]["sample"]
+    # the GPU arm builds its `config` with the same function, so the two arms'
+    # lines name the same workload with the same keys
+    sys.path.insert(0, ROOT)
+    import bench
+    from moe_synth import get_config
+    assert j["config"] == bench.run_config(get_config("tiny_fp32"), 0, 1)
+
+
+def test_default_workload_is_the_large_expert_layer():
+    sys.path.insert(0, ROOT)
+    import bench
+    import inspect
+    src = inspect.getsource(bench.main)
+    assert 'ap.add_argument("--config", default="large_e")' in src
 
 
 def test_reference_other_ranks_exit_quietly():
