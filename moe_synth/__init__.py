@@ -36,6 +36,7 @@ from __future__ import annotations
 
 import json
 import os
+from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass, replace
 from typing import Dict, Optional
 
@@ -225,8 +226,14 @@ def make_experts(shape: MoEShape, seed: int):
     wg = torch.empty(N, F, d, dtype=dt)
     wu = torch.empty(N, F, d, dtype=dt)
     wd = torch.empty(N, d, F, dtype=dt)
-    for e in range(N):
+
+    def draw(e):
         wg[e], wu[e], wd[e] = make_expert(shape, seed, e)
+
+    # every expert has its own generator, so drawing them on several threads
+    # gives the same tensors as drawing them in order
+    with ThreadPoolExecutor(max(1, min(16, os.cpu_count() or 1))) as ex:
+        list(ex.map(draw, range(N)))
     _expert_cache[key] = (wg, wu, wd)
     return wg, wu, wd
 

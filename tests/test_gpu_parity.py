@@ -43,7 +43,65 @@ SMALL = [
 ]
 
 
+def stratified_rows(r_counts, r_offsets, N, seed, n_sub=48, n_full=2):
+    """Rows of y_perm (dispatch order) to check at sizes where the oracle
+    cannot compute them all. The expert GEMMs cut an expert's segment into
+    token tiles of 64, 128 or 256 rows (the batch size decides), and a CTA pair
+    splits each tile in halves. The sample holds:
+      * for every touched expert, the first and last row of its segment and
+        its last partial 256-row tile (whole up to 16 rows, else its first and
+        last 8);
+      * for n_sub seeded experts, the first and last row of every 128- and
+        256-row tile and the last partial 128-row tile (same rule);
+      * every row of the first and last 256-row tiles of the most loaded
+        expert (the Zipf-hot one under skewed routing) and of n_full seeded
+        others.
+    """
+    rows = set()
+    touched = np.nonzero(r_counts[:N])[0]
+    rng = np.random.default_rng(seed)
+    sub = {int(e) for e in rng.choice(touched, size=min(n_sub, touched.size), replace=False)}
+
+    def tail_of(o, n, tile):
+        t = list(range(o + ((n - 1) // tile) * tile, o + n))
+        return t if len(t) <= 16 else t[:8] + t[-8:]
+
+    for e in touched:
+        o, n = int(r_offsets[e]), int(r_counts[e])
+        rows.update((o, o + n - 1))
+        rows.update(tail_of(o, n, 256))
+        if int(e) in sub:
+            for tile in (128, 256):
+                for t in range((n + tile - 1) // tile):
+                    rows.update((o + t * tile, min(o + n, o + (t + 1) * tile) - 1))
+            rows.update(tail_of(o, n, 128))
+    hot = int(touched[np.argmax(r_counts[touched])])
+    full = {hot} | {int(e) for e in rng.choice(touched, size=min(n_full, touched.size),
+                                               replace=False)}
+    for e in sorted(full):
+        o, n = int(r_offsets[e]), int(r_counts[e])
+        rows.update(range(o, o + min(n, 256)))
+        rows.update(range(o + ((n - 1) // 256) * 256, o + n))
+    return np.array(sorted(rows), dtype=np.int64)
+
+
+def stratified_tokens(rows, r_row_token, ref_idx, N, T, seed, n_tok=48):
+    """Tokens whose whole layer output is checked: up to n_tok of the tokens
+    behind the stratified rows, 8 seeded others, and up to 8 tokens that send
+    a slot to a zero expert (the identity term)."""
+    rng = np.random.default_rng(seed + 7)
+    behind = np.unique(r_row_token[rows])
+    pick = set(rng.choice(behind, size=min(n_tok, behind.size), replace=False).tolist())
+    pick |= set(rng.choice(T, size=min(8, T), replace=False).tolist())
+    zero_tok = np.nonzero((ref_idx >= N).any(axis=1))[0]
+    if zero_tok.size:
+        pick |= set(rng.choice(zero_tok, size=min(8, zero_tok.size), replace=False).tolist())
+    return np.array(sorted(pick), dtype=np.int64)
+
+
 def run_staged_and_fused(sh: MoEShape, seed: int, sample=None, s=None):
+    """sample=None checks every row and token; sample="strat" checks the
+    stratified rows and tokens above."""
     inp = make_inputs(sh, seed)
     ls = layer_shape(sh, s)
     scale = ls.routed_scale
@@ -85,8 +143,7 @@ def run_staged_and_fused(sh: MoEShape, seed: int, sample=None, s=None):
                             d_inp.w_gate, d_inp.w_up, d_inp.w_down, ws)
     torch.cuda.synchronize()
     row_expert = np.repeat(np.arange(N), r_counts[:N]).astype(np.int32)
-    rows = np.arange(R) if sample is None else np.unique(
-        np.random.default_rng(seed).choice(R, size=min(sample, R), replace=False))
+    rows = np.arange(R) if sample is None else stratified_rows(r_counts, r_offsets, N, seed)
     if R > 0:
         y_ref = oracle.expert_rows(inp.w_gate, inp.w_up, inp.w_down, row_expert[rows],
                                    x_perm_ref[torch.from_numpy(rows).long()])
@@ -95,8 +152,8 @@ def run_staged_and_fused(sh: MoEShape, seed: int, sample=None, s=None):
         assert err <= OUT_RTOL_RMS, f"expert rows: max err {err:.3e} x rms"
 
     # ---- combine, fed the oracle's gates and expert outputs (rounded to fp32)
-    tok = np.arange(T) if sample is None else np.unique(
-        np.random.default_rng(seed + 7).choice(T, size=min(sample, T), replace=False))
+    tok = np.arange(T) if sample is None else stratified_tokens(rows, r_row_token, ref_idx,
+                                                                N, T, seed)
     if sample is None and R > 0:
         y_all = oracle.expert_rows(inp.w_gate, inp.w_up, inp.w_down, row_expert,
                                    x_perm_ref[:R])
@@ -175,16 +232,25 @@ def test_decode_full(seed):
 
 
 def test_prefill_full_sampled():
-    run_staged_and_fused(CONFIGS["prefill"], 0, sample=48)
+    run_staged_and_fused(CONFIGS["prefill"], 0, sample="strat")
 
 
+# the large-expert layer and the sweep share one set of expert weights (d=6144,
+# 256 experts of width 2048), drawn once while these tests run back to back
 def test_large_e_full_sampled():
-    info = run_staged_and_fused(CONFIGS["large_e"], 0, sample=24)
+    info = run_staged_and_fused(CONFIGS["large_e"], 0, sample="strat")
     sh = CONFIGS["large_e"]
     zero_share = 1.0 - info["R"] / (sh.T * sh.top_k)
     assert 0.29 <= zero_share <= 0.31
 
 
+@pytest.mark.parametrize("routing", ["uniform", "zipf"])
 @pytest.mark.parametrize("T", [1, 8, 64])
-def test_sweep_small_T(T):
-    run_staged_and_fused(get_config(f"sweep_uniform_T{T}"), 0)
+def test_sweep_small_T(T, routing):
+    run_staged_and_fused(get_config(f"sweep_{routing}_T{T}"), 0)
+
+
+@pytest.mark.parametrize("routing", ["uniform", "zipf"])
+@pytest.mark.parametrize("T", [512, 4096, 32768])
+def test_sweep_large_T_sampled(T, routing):
+    run_staged_and_fused(get_config(f"sweep_{routing}_T{T}"), 0, sample="strat")
