@@ -412,7 +412,7 @@ def run_gpu(args, sh):
         b_disp = 2 * Tk * 4 + Tk * 4 * 2 + 2 * R * sh.d * es
         b_ffn = U * 3 * sh.ffn * sh.d * es
         n_zero_tok = int(((idx >= sh.n_routed).any(dim=1)).sum())
-        b_comb = R * sh.d * 4 + n_zero_tok * sh.d * es + sh.T * sh.d * es + Tk * 12
+        b_comb = R * sh.d * es + n_zero_tok * sh.d * es + sh.T * sh.d * es + Tk * 12
         flops_ffn = 6.0 * R * sh.d * sh.ffn
         hbm = pk["hbm_gbs"]
 

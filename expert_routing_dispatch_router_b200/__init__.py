@@ -240,7 +240,7 @@ def dispatch(shape: LayerShape, x, topk_idx, ws, stream=None):
 
 def expert_ffn(shape: LayerShape, x_perm, offsets, w_gate, w_up, w_down, ws,
                y_perm=None, stream=None):
-    """-> y_perm [T*k, d] float32 (rows >= R untouched)."""
+    """-> y_perm [T*k, d] in the activation dtype (rows >= R untouched)."""
     T, k, d, F, N = shape.T, shape.top_k, shape.d, shape.ffn, shape.n_routed
     _need(x_perm, "x_perm", shape.act_dtype, (T * k, d))
     _need(offsets, "offsets", torch.int32, (N + 1,))
@@ -248,8 +248,8 @@ def expert_ffn(shape: LayerShape, x_perm, offsets, w_gate, w_up, w_down, ws,
                          ("w_down", w_down, (N, d, F))):
         _need(w, name, shape.act_dtype, shp)
     if y_perm is None:
-        y_perm = torch.empty(T * k, d, dtype=torch.float32, device=x_perm.device)
-    _need(y_perm, "y_perm", torch.float32, (T * k, d))
+        y_perm = torch.empty(T * k, d, dtype=shape.act_dtype, device=x_perm.device)
+    _need(y_perm, "y_perm", shape.act_dtype, (T * k, d))
     st = lib().moe_expert_ffn(ctypes.byref(shape.c()), _ptr(x_perm), _ptr(offsets),
                               _ptr(w_gate), _ptr(w_up), _ptr(w_down), _ptr(y_perm),
                               *_ws(ws), _stream(stream))
@@ -261,7 +261,7 @@ def combine(shape: LayerShape, x, y_perm, topk_idx, topk_gate, slot_row, out=Non
             stream=None):
     T, k, d = shape.T, shape.top_k, shape.d
     _need(x, "x", shape.act_dtype, (T, d))
-    _need(y_perm, "y_perm", torch.float32, (T * k, d))
+    _need(y_perm, "y_perm", shape.act_dtype, (T * k, d))
     _need(topk_idx, "topk_idx", torch.int32, (T, k))
     _need(topk_gate, "topk_gate", torch.float32, (T, k))
     _need(slot_row, "slot_row", torch.int32, (T * k,))

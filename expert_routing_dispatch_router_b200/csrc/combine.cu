@@ -10,10 +10,11 @@
 //   out[t] = s * sum_{j: idx<N} gate[t,j] * y_perm[slot_row[t,j]]
 //              + sum_{j: idx>=N} gate[t,j] * x[t]
 //
-// y_perm is fp32. Both sums run in fp32 in slot order j = 0..k-1 and the
-// result is rounded once, so the output does not depend on thread timing.
-// When the fused layer split the down GEMM's contraction (tiny batches), each
-// row of y holds ysplit partial rows, added in split order first: the same
+// y_perm is in the activation type, like x and out. Both sums run in fp32 in
+// slot order j = 0..k-1 and the result is rounded once, so the output does not
+// depend on thread timing. When the fused layer split the down GEMM's
+// contraction (tiny batches), y holds ysplit fp32 partial rows per slot row:
+// they are added in split order and rounded to the activation type, the same
 // arithmetic as reducing them into y_perm and combining that.
 // Grid: one block row per token, 16-byte vectors along d.
 #include "moe_internal.cuh"
@@ -60,9 +61,19 @@ struct Vec<float> {
   }
 };
 
+// the value a stored activation would have: v rounded to AT
+template <typename AT>
+__device__ __forceinline__ float round_to(float v);
+template <>
+__device__ __forceinline__ float round_to<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ float round_to<__nv_bfloat16>(float v) {
+  return __bfloat162float(__float2bfloat16_rn(v));
+}
+
 template <typename AT>
 __global__ void __launch_bounds__(128)
-    combine_kernel(const AT* __restrict__ x, const float* __restrict__ y,
+    combine_kernel(const AT* __restrict__ x, const void* __restrict__ y_any,
                    const int32_t* __restrict__ idx,
                    const float* __restrict__ gate,
                    const int32_t* __restrict__ slot_row, AT* __restrict__ out,
@@ -93,29 +104,44 @@ __global__ void __launch_bounds__(128)
   // slots four at a time: the y loads of a group are issued together, then
   // added in slot order
   for (int j0 = 0; j0 < k; j0 += 4) {
-    const float* yr[4];
+    int64_t ro[4];  // offset of each slot's y row, -1 for none
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const int j = j0 + q;
       const int r = j < k && !s_zero[j] ? s_row[j] : -1;
-      yr[q] = r >= 0 ? y + (int64_t)r * ysplit * d + col : nullptr;
+      ro[q] = r >= 0 ? (int64_t)r * ysplit * d + col : -1;
     }
     float yv[4][V];
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-      if (yr[q] != nullptr) {
-#pragma unroll
-        for (int i = 0; i < V; i += 4) Vec<float>::load(yr[q] + i, yv[q] + i);
-      }
-    // split partials of each slot's row, added in split order (none for plain y)
-    for (int c = 1; c < ysplit; ++c) {
+    if (ysplit == 1) {
+      const AT* y = static_cast<const AT*>(y_any);
 #pragma unroll
       for (int q = 0; q < 4; ++q)
-        if (yr[q] != nullptr) {
+        if (ro[q] >= 0) Vec<AT>::load(y + ro[q], yv[q]);
+    } else {
+      // fp32 split partials of each slot's row, added in split order, then
+      // rounded as a stored y_perm row would be
+      const float* y = static_cast<const float*>(y_any);
 #pragma unroll
-          for (int i = 0; i < V; i += 4) Vec<float>::load(yr[q] + (int64_t)c * d + i, v + i);
+      for (int q = 0; q < 4; ++q)
+        if (ro[q] >= 0) {
 #pragma unroll
-          for (int i = 0; i < V; ++i) yv[q][i] += v[i];
+          for (int i = 0; i < V; i += 4) Vec<float>::load(y + ro[q] + i, yv[q] + i);
+        }
+      for (int c = 1; c < ysplit; ++c) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (ro[q] >= 0) {
+#pragma unroll
+            for (int i = 0; i < V; i += 4) Vec<float>::load(y + ro[q] + (int64_t)c * d + i, v + i);
+#pragma unroll
+            for (int i = 0; i < V; ++i) yv[q][i] += v[i];
+          }
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (ro[q] >= 0) {
+#pragma unroll
+          for (int i = 0; i < V; ++i) yv[q][i] = round_to<AT>(yv[q][i]);
         }
     }
 #pragma unroll
@@ -126,7 +152,7 @@ __global__ void __launch_bounds__(128)
       if (s_zero[j]) {
 #pragma unroll
         for (int i = 0; i < V; ++i) zacc[i] = fmaf(g, xv[i], zacc[i]);
-      } else if (yr[q] != nullptr) {
+      } else if (ro[q] >= 0) {
 #pragma unroll
         for (int i = 0; i < V; ++i) racc[i] = fmaf(g, yv[q][i], racc[i]);
       }
@@ -149,12 +175,12 @@ cudaError_t launch_combine(const Shape& sh, const void* x, const void* y_perm,
   dim3 grid((unsigned)sh.T, (unsigned)((vecs + threads - 1) / threads));
   if (sh.bf16)
     launch_pdl(combine_kernel<__nv_bfloat16>, grid, dim3(threads), 0, st,
-               static_cast<const __nv_bfloat16*>(x), static_cast<const float*>(y_perm),
+               static_cast<const __nv_bfloat16*>(x), y_perm,
                idx, gate, slot_row, static_cast<__nv_bfloat16*>(out), sh.d, (int)sh.N,
                (int)sh.k, sh.s, ysplit);
   else
     launch_pdl(combine_kernel<float>, grid, dim3(threads), 0, st,
-               static_cast<const float*>(x), static_cast<const float*>(y_perm), idx,
+               static_cast<const float*>(x), y_perm, idx,
                gate, slot_row, static_cast<float*>(out), sh.d, (int)sh.N, (int)sh.k,
                sh.s, ysplit);
   return cudaGetLastError();

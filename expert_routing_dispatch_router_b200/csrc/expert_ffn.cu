@@ -141,7 +141,7 @@ struct Cfg {
 struct GemmArgs {
   const int32_t* offsets;     // [N+1] row offsets per expert
   const int32_t* tile_start;  // [N+1] token-tile prefix per expert
-  void* out;                  // [rows_cap, out_cols]: bf16 h or fp32 y
+  void* out;                  // [rows_cap, out_cols]: bf16 h, bf16 y or fp32 rows
   int32_t* err;               // workspace error word
   int N;
   int num_kb;    // contraction length / BK
@@ -165,6 +165,9 @@ struct GemmArgs {
   // CTA pairs: units are handed out in order from this counter (zeroed with
   // the tile plan before the launch)
   int* unit_counter = nullptr;
+  // Down GEMM: output rows in bf16 (the expert outputs y_perm) instead of
+  // fp32 (the router's logits and split-contraction partials)
+  bool out_bf16 = false;
 };
 
 struct Unit {
@@ -531,10 +534,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c0 = 32 * eh; c0 < un.n_mma; c0 += 64) {
           float g[32];
           ptx::tmem_ld32(tb + c0, g);
-          float* outp = static_cast<float*>(args.out) + obase;
+          if (args.out_bf16) {
+            __nv_bfloat16* outp = static_cast<__nv_bfloat16*>(args.out) + obase;
 #pragma unroll
-          for (int c = 0; c < 32; ++c)
-            if (c0 + c < un.n_valid) outp[(int64_t)(c0 + c) * args.out_cols] = g[c];
+            for (int c = 0; c < 32; ++c)
+              if (c0 + c < un.n_valid)
+                outp[(int64_t)(c0 + c) * args.out_cols] = __float2bfloat16_rn(g[c]);
+          } else {
+            float* outp = static_cast<float*>(args.out) + obase;
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+              if (c0 + c < un.n_valid) outp[(int64_t)(c0 + c) * args.out_cols] = g[c];
+          }
         }
         release();
       }
@@ -587,11 +598,12 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// y[r, :] = sum_c part[r][c][:] in order c = 0..s-1, for the routed rows r < R
-// (the down GEMM's split partials, [row][c][d] fp32).
+// y[r, :] = bf16(sum_c part[r][c][:]), the sum in fp32 in order c = 0..s-1,
+// for the routed rows r < R (the down GEMM's split partials, [row][c][d]).
 __global__ void __launch_bounds__(256)
     split_reduce_kernel(const float* __restrict__ part, int s, int64_t d,
-                        const int32_t* __restrict__ offsets, int N, float* __restrict__ y) {
+                        const int32_t* __restrict__ offsets, int N,
+                        __nv_bfloat16* __restrict__ y) {
   griddep_wait();
   griddep_launch_dependents();
   const int64_t R = offsets[N];
@@ -605,7 +617,12 @@ __global__ void __launch_bounds__(256)
       const float4 w = *reinterpret_cast<const float4*>(p + (int64_t)c * d);
       v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
     }
-    *reinterpret_cast<float4*>(y + r * d + col) = v;
+    const __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y);
+    const __nv_bfloat162 b = __floats2bfloat162_rn(v.z, v.w);
+    uint2 o;
+    o.x = *reinterpret_cast<const uint32_t*>(&a);
+    o.y = *reinterpret_cast<const uint32_t*>(&b);
+    *reinterpret_cast<uint2*>(y + r * d + col) = o;
   }
 }
 
@@ -901,14 +918,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         swiglu_epilogue<BN / 64>(tb, BN, eh, n_pair, un.n_valid,
                                  static_cast<__nv_bfloat16*>(args.out) + obase, args.out_cols,
                                  release);
-      } else {
+      } else {  // pairs run only the expert GEMMs: y in bf16
+        __nv_bfloat16* outp = static_cast<__nv_bfloat16*>(args.out) + obase;
         for (int c0 = 32 * eh; c0 < n_pair; c0 += 64) {
           float g[32];
           ptx::tmem_ld32(tb + c0, g);
-          float* outp = static_cast<float*>(args.out) + obase;
 #pragma unroll
           for (int c = 0; c < 32; ++c)
-            if (c0 + c < un.n_valid) outp[(int64_t)(c0 + c) * args.out_cols] = g[c];
+            if (c0 + c < un.n_valid)
+              outp[(int64_t)(c0 + c) * args.out_cols] = __float2bfloat16_rn(g[c]);
         }
         release();
       }
@@ -1087,11 +1105,11 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// y[r, n] = h[r] . w_down[e, n]   (y kept in fp32)
+// y[r, n] = h[r] . w_down[e, n]   (fp32 sum, stored in the activation type)
 template <typename AT>
 __global__ void __launch_bounds__(256)
     ffn_down_simt_kernel(const AT* __restrict__ h, const int32_t* __restrict__ offsets,
-                         int N, const AT* __restrict__ wd, float* __restrict__ y,
+                         int N, const AT* __restrict__ wd, AT* __restrict__ y,
                          int64_t d, int64_t F) {
   griddep_wait();
   griddep_launch_dependents();
@@ -1107,7 +1125,7 @@ __global__ void __launch_bounds__(256)
     float acc = 0.f;
     for (int64_t f = lane; f < F; f += 32) acc = fmaf(to_f32(dr[f]), to_f32(hr[f]), acc);
     acc = warp_sum<AT>(acc);
-    if (lane == 0) y[r * d + n] = acc;
+    if (lane == 0) y[r * d + n] = from_f32<AT>(acc);
   }
 }
 
@@ -1123,7 +1141,7 @@ cudaError_t launch_simt(const Shape& sh, const void* x_perm, const int32_t* offs
   if (e != cudaSuccess) return e;
   return launch_pdl(ffn_down_simt_kernel<AT>, dim3(blocks), dim3(256), 0, st,
                     static_cast<const AT*>(h), offsets, (int)sh.N,
-                    static_cast<const AT*>(wd), static_cast<float*>(y), sh.d, sh.F);
+                    static_cast<const AT*>(wd), static_cast<AT*>(y), sh.d, sh.F);
 }
 
 }  // namespace
@@ -1273,6 +1291,7 @@ cudaError_t launch_expert_ffn(const Shape& sh, const void* x_perm,
     dp.unit_counter = tile_start + 2 * sh.N + 3;
     dp.tile_start = tile_start + sh.N + 1;
     dp.out = y_perm;
+    dp.out_bf16 = true;
     dp.num_kb = (int)(sh.F / BK);
     dp.out_cols = (int)sh.d;
     dp.a_rows = (int)sh.d;
@@ -1307,6 +1326,7 @@ cudaError_t launch_expert_ffn(const Shape& sh, const void* x_perm,
   dn.part = nullptr;
   dn.tile_start = tile_start + sh.N + 1;
   dn.out = sd > 1 ? static_cast<void*>(part) : y_perm;
+  dn.out_bf16 = sd == 1;  // split partials stay fp32 until they are added
   dn.num_kb = (int)(sh.F / BK);
   dn.out_cols = (int)sh.d * sd;  // split c writes columns [c d, (c + 1) d)
   dn.m_tiles = (int)(sh.d / BM) * sd;
@@ -1319,7 +1339,7 @@ cudaError_t launch_expert_ffn(const Shape& sh, const void* x_perm,
   if (e != cudaSuccess || sd == 1 || leave_y_split) return e;
   return launch_pdl(split_reduce_kernel, dim3(fix_blocks), dim3(256), 0, st,
                     static_cast<const float*>(part), sd, sh.d, offsets, (int)sh.N,
-                    static_cast<float*>(y_perm));
+                    static_cast<__nv_bfloat16*>(y_perm));
 }
 
 }  // namespace moe

@@ -43,7 +43,7 @@ WsLayout ws_layout(const Shape& sh) {
   L.tile_start = take((2 * (size_t)(sh.N + 1) + 2) * sizeof(int32_t));
   L.x_perm = take(Tk * sh.d * sh.es);
   L.h = take(Tk * sh.F * sh.es);
-  L.y_perm = take(Tk * sh.d * sizeof(float));
+  L.y_perm = take(Tk * sh.d * sh.es);
   L.ffn_part = take(sh.N > 0 ? (size_t)expert_ffn_part_floats(sh) * sizeof(float) : 0);
   L.x_stage = take((size_t)sh.T * sh.d * sh.es);
   L.out_stage = take((size_t)sh.T * sh.d * sh.es);

@@ -42,7 +42,7 @@ struct WsLayout {
                        // the CTA-pair GEMMs' unit counters
   size_t x_perm;       // act   [T*k, d]
   size_t h;            // act   [T*k, F]
-  size_t y_perm;       // float [T*k, d]
+  size_t y_perm;       // act [T*k, d]
   size_t ffn_part;     // float split-contraction partials of the expert GEMMs
                        // (tiny batches only; else empty)
   size_t x_stage;      // act   [T, d]   (host-buffer entry point)

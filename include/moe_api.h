@@ -27,10 +27,9 @@
  *    are dense row-major. Every pointer must be 16-byte aligned. The device
  *    pointers of a call must all be memory of the current CUDA device, the
  *    one `stream` belongs to: kernels run there and read them directly.
- *  - act_dtype is the type of x, out, the expert weights and x_perm:
- *    MOE_F32 (float) or MOE_BF16 (bfloat16). w_router, bias, topk_gate and
- *    the expert outputs y_perm are always float; indices are int32. (y_perm
- *    stays fp32 so that only h and out are rounded to bf16.)
+ *  - act_dtype is the type of x, out, the expert weights, x_perm, h and the
+ *    expert outputs y_perm: MOE_F32 (float) or MOE_BF16 (bfloat16).
+ *    w_router, bias and topk_gate are always float; indices are int32.
  *  - Every call is asynchronous on `stream` (0 = legacy default stream) and
  *    issues no host synchronisation, so a sequence of calls can be captured
  *    in a CUDA graph.
@@ -130,10 +129,10 @@ moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x,
  * Model card, "Mixture of experts": expert dim; activation taken as SwiGLU.
  *  x_perm  [T*k, d] act_dtype;  offsets [N+1] int32 (as from moe_dispatch)
  *  w_gate, w_up [N, F, d] act_dtype;  w_down [N, d, F] act_dtype
- *  y_perm  [T*k, d] float: y_perm[r] = y_e(x_perm[r]) for r < R, e the
+ *  y_perm  [T*k, d] act_dtype: y_perm[r] = y_e(x_perm[r]) for r < R, e the
  *          expert owning row r; rows >= R are left as they were.
  *  bf16 with d and F multiples of 128 runs on tcgen05 tensor cores (fp32
- *  accumulation in TMEM, h rounded to bf16); other shapes and f32 run on a
+ *  accumulation in TMEM, h and y rounded to bf16); other shapes and f32 run on a
  *  CUDA-core path with fp32 accumulation. */
 moe_status_t moe_expert_ffn(const moe_config_t* cfg, const void* x_perm,
                             const int32_t* offsets, const void* w_gate,
@@ -144,7 +143,7 @@ moe_status_t moe_expert_ffn(const moe_config_t* cfg, const void* x_perm,
  * summed in fp32 in slot order j = 0..k-1 and rounded once (deterministic).
  * Ascend deployment article, "底层定制算子深度优化" (Combine operator);
  * model card, "Routed scaling factor".
- *  x [T, d], out [T, d] act_dtype; y_perm [T*k, d] float; topk_idx,
+ *  x [T, d], out [T, d], y_perm [T*k, d] act_dtype; topk_idx,
  *  topk_gate, slot_row as above. */
 moe_status_t moe_combine(const moe_config_t* cfg, const void* x,
                          const void* y_perm, const int32_t* topk_idx,
