@@ -99,7 +99,13 @@ def test_pairs_no_routed_slots():
                                      ((255, 0, 0, 1, 17, 384, 64), 384),
                                      # T > 1024: both GEMMs run on CTA pairs
                                      ((1, 31, 32, 33, 255, 256, 257, 300), 512),
-                                     ((0, 600, 0, 1, 520), 512)])
+                                     ((0, 600, 0, 1, 520), 512),
+                                     # T > 1024 with F = 384 (not a multiple of
+                                     # 256): single-CTA GEMMs with 256-token
+                                     # tiles, segments around 1 and 2 tiles and
+                                     # one expert cut into 33 tiles
+                                     ((287, 288, 289, 511, 512, 513, 1025), 384),
+                                     ((8200, 3, 0, 700), 384)])
 def test_expert_segments_around_tile_size(sizes, F):
     """moe_expert_ffn on crafted segments: offsets give exactly these rows per
     expert; rows are random bf16; checked row by row against the oracle."""
