@@ -5,9 +5,21 @@
 #include <math.h>
 #include <string.h>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "moe_internal.cuh"
 
 namespace moe {
+
+// NVTX range over a host-side scope: each call and each stage of the fused
+// layer shows up by name in a profiler's timeline (header-only NVTX; without
+// a profiler attached a push or pop is one check of a null hook).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 static size_t align_up(size_t v) {
   return (v + kWsAlign - 1) / kWsAlign * kWsAlign;
@@ -117,9 +129,12 @@ moe_status_t run_layer(const Shape& sh, const void* x, const float* w_router,
   int32_t* offsets = at<int32_t>(ws, L.offsets);
   void* x_perm = at<void>(ws, L.x_perm);
   void* y_perm = at<void>(ws, L.y_perm);
-  cudaError_t e = launch_router(sh, x, w_router, bias, at<float>(ws, L.logits), idx,
-                                gate, nullptr, nullptr, at<void>(ws, L.planes),
-                                at<int32_t>(ws, L.router_plan), err, st);
+  cudaError_t e;
+  {
+    NvtxRange r("moe.route");
+    e = launch_router(sh, x, w_router, bias, at<float>(ws, L.logits), idx, gate, nullptr,
+                      nullptr, at<void>(ws, L.planes), at<int32_t>(ws, L.router_plan), err, st);
+  }
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   // where the gate/up GEMM gathers token rows itself, x_perm is never written
   const bool gather = expert_ffn_gathers(sh);
@@ -129,18 +144,25 @@ moe_status_t run_layer(const Shape& sh, const void* x, const float* w_router,
   expert_ffn_tiles(sh, &tgu, &tdn);
   int32_t* row_token = at<int32_t>(ws, L.row_token);
   int32_t* tile_start = at<int32_t>(ws, L.tile_start);
-  e = launch_dispatch(sh, x, idx, at<int32_t>(ws, L.chunk_base),
-                      counts ? counts : at<int32_t>(ws, L.counts), offsets, row_token,
-                      slot_row, gather ? nullptr : x_perm, err, st, plan ? tile_start : nullptr,
-                      tgu, tdn);
+  {
+    NvtxRange r("moe.dispatch");
+    e = launch_dispatch(sh, x, idx, at<int32_t>(ws, L.chunk_base),
+                        counts ? counts : at<int32_t>(ws, L.counts), offsets, row_token,
+                        slot_row, gather ? nullptr : x_perm, err, st,
+                        plan ? tile_start : nullptr, tgu, tdn);
+  }
   if (e != cudaSuccess) return MOE_ERR_CUDA;
   // with a split down GEMM, the combine adds its partials itself
   const int ysplit = sh.N > 0 ? expert_ffn_split(sh, false) : 1;
   float* part = at<float>(ws, L.ffn_part);
-  e = launch_expert_ffn(sh, x_perm, offsets, w_gate, w_up, w_down, at<void>(ws, L.h),
-                        y_perm, tile_start, err, st, gather ? x : nullptr,
-                        gather ? row_token : nullptr, plan, part, true);
+  {
+    NvtxRange r("moe.expert_ffn");
+    e = launch_expert_ffn(sh, x_perm, offsets, w_gate, w_up, w_down, at<void>(ws, L.h),
+                          y_perm, tile_start, err, st, gather ? x : nullptr,
+                          gather ? row_token : nullptr, plan, part, true);
+  }
   if (e != cudaSuccess) return MOE_ERR_CUDA;
+  NvtxRange r("moe.combine");
   e = launch_combine(sh, x, ysplit > 1 ? static_cast<void*>(part) : y_perm, idx, gate,
                      slot_row, out, st, ysplit);
   return cuda_status(e);
@@ -165,6 +187,7 @@ moe_status_t moe_route(const moe_config_t* cfg, const void* x, const float* w_ro
                        const float* bias, float* logits, int32_t* topk_idx,
                        float* topk_gate, uint8_t* flags, void* ws, size_t ws_bytes,
                        moe_stream_t stream) {
+  NvtxRange range("moe_route");
   Shape sh;
   moe_status_t s = make_shape(cfg, &sh);
   if (s != MOE_OK) return s;
@@ -185,6 +208,7 @@ moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t*
                           int32_t* counts, int32_t* offsets, int32_t* row_token,
                           int32_t* slot_row, void* x_perm, void* ws, size_t ws_bytes,
                           moe_stream_t stream) {
+  NvtxRange range("moe_dispatch");
   Shape sh;
   moe_status_t s = make_shape(cfg, &sh);
   if (s != MOE_OK) return s;
@@ -204,6 +228,7 @@ moe_status_t moe_expert_ffn(const moe_config_t* cfg, const void* x_perm,
                             const int32_t* offsets, const void* w_gate, const void* w_up,
                             const void* w_down, void* y_perm, void* ws, size_t ws_bytes,
                             moe_stream_t stream) {
+  NvtxRange range("moe_expert_ffn");
   Shape sh;
   moe_status_t s = make_shape(cfg, &sh);
   if (s != MOE_OK) return s;
@@ -224,6 +249,7 @@ moe_status_t moe_expert_ffn(const moe_config_t* cfg, const void* x_perm,
 moe_status_t moe_combine(const moe_config_t* cfg, const void* x, const void* y_perm,
                          const int32_t* topk_idx, const float* topk_gate,
                          const int32_t* slot_row, void* out, moe_stream_t stream) {
+  NvtxRange range("moe_combine");
   Shape sh;
   moe_status_t s = make_shape(cfg, &sh);
   if (s != MOE_OK) return s;
@@ -240,6 +266,7 @@ moe_status_t moe_layer_forward(const moe_config_t* cfg, const void* x,
                                const void* w_gate, const void* w_up, const void* w_down,
                                void* out, int32_t* counts, void* ws, size_t ws_bytes,
                                moe_stream_t stream) {
+  NvtxRange range("moe_layer_forward");
   Shape sh;
   moe_status_t s = make_shape(cfg, &sh);
   if (s != MOE_OK) return s;
@@ -260,6 +287,7 @@ moe_status_t moe_layer_forward_host(const moe_config_t* cfg, const void* x_host,
                                     const void* w_down, void* out_host,
                                     int32_t* counts_host, void* ws, size_t ws_bytes,
                                     moe_stream_t stream) {
+  NvtxRange range("moe_layer_forward_host");
   Shape sh;
   moe_status_t s = make_shape(cfg, &sh);
   if (s != MOE_OK) return s;
@@ -291,6 +319,7 @@ moe_status_t moe_layer_forward_host(const moe_config_t* cfg, const void* x_host,
 moe_status_t moe_bias_pid_update(const moe_config_t* cfg, const int32_t* counts,
                                  float* bias, double* state,
                                  const moe_pid_params_t* params, moe_stream_t stream) {
+  NvtxRange range("moe_bias_pid_update");
   Shape sh;
   moe_status_t s = make_shape(cfg, &sh);
   if (s != MOE_OK) return s;
