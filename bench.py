@@ -484,25 +484,35 @@ def run_gpu(args, sh):
     replicas.finalize(info)
 
 
-def main():
+def make_parser():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--config", default="large_e")
+    ap.add_argument("--config", default="large_e",
+                    help="workload name; on one GPU a comma-separated list runs each in "
+                         "turn in one process (one JSON line each), e.g. the sweep points")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-tokens", type=int, default=0,
                     help="tokens per reference step (default: one per host thread)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    args = ap.parse_args()
+    return ap
+
+
+def main():
+    args = make_parser().parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    sh = get_config(args.config)
-    if args.impl == "reference":
-        run_reference(args, sh)
-    else:
-        run_gpu(args, sh)
+    names = [n for n in args.config.split(",") if n]
+    if len(names) > 1 and (args.impl == "reference" or int(os.environ.get("WORLD_SIZE", "1")) > 1):
+        raise SystemExit("a list of workloads runs on one GPU, ours only")
+    for name in names:
+        sh = get_config(name)
+        if args.impl == "reference":
+            run_reference(args, sh)
+        else:
+            run_gpu(args, sh)
 
 
 if __name__ == "__main__":

@@ -45,9 +45,8 @@ def test_reference_line_has_the_contract_keys():
 def test_default_workload_is_the_large_expert_layer():
     sys.path.insert(0, ROOT)
     import bench
-    import inspect
-    src = inspect.getsource(bench.main)
-    assert 'ap.add_argument("--config", default="large_e")' in src
+    args = bench.make_parser().parse_args([])
+    assert args.config == "large_e" and args.gpus == 1 and args.impl == "ours"
 
 
 def test_reference_other_ranks_exit_quietly():
