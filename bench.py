@@ -446,7 +446,8 @@ def run_gpu(args, sh):
         if flops_ffn / (pk["bf16_tflops"] * 1e12) > b_ffn / (pk["hbm_gbs"] * 1e9):
             ach = flops_ffn / t_ffn / 1e9
             roof = {"bound": "tensor", "achieved": ach, "peak": pk["bf16_tflops"],
-                    "unit": "TFLOP/s", "frac": ach / pk["bf16_tflops"], "traffic": None,
+                    "unit": "TFLOP/s", "frac": ach / pk["bf16_tflops"],
+                    "traffic": measured_traffic(sh.name, U),
                     "kernel": "moe_expert_ffn: grouped GEMM gate/up + down (+ plan)",
                     "algorithmic_flops": flops_ffn,
                     "peak_source": pk["source"] + " bf16_tflops (burst cuBLAS GEMM)"}

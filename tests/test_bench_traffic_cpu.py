@@ -49,3 +49,10 @@ def test_committed_record_is_well_formed():
     entry = rec["decode"]
     assert entry["dram_bytes_per_touched_expert"] > 0
     assert len(entry["source_digest"]) == 16
+
+
+def test_headline_workload_traffic_record_is_current():
+    # the committed capture of the CTA-pair GEMMs was taken on the current
+    # expert-GEMM sources, so the default bench line reports its DRAM traffic
+    t = bench.measured_traffic("large_e", 256)
+    assert t is not None and 19.3e9 < t < 30e9
