@@ -33,7 +33,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from moe_synth import get_config, make_inputs, torch_dtype  # noqa: E402
+from moe_synth import get_config, make_inputs, make_tokens, torch_dtype  # noqa: E402
 
 METRIC = "MoE-layer tokens/s; grouped-GEMM % bf16 TC peak; router/dispatch/combine GB/s"
 
@@ -277,7 +277,10 @@ def run_gpu(args, sh):
     stream = torch.cuda.current_stream()
     pk = peaks()
 
-    inp = make_inputs(sh, replicas.batch_seed(args.seed, info))
+    # one model (router and expert weights of the base seed); every rank
+    # routes its own batch of tokens
+    inp = make_inputs(sh, args.seed)
+    inp.x = make_tokens(sh, replicas.batch_seed(args.seed, info))
     d = inp.to(dev)
     ls = moe.LayerShape(sh.T, sh.d, sh.n_routed, sh.n_zero, sh.top_k, sh.ffn,
                         torch_dtype(sh.act_dtype), sh.routed_scale)

@@ -177,10 +177,16 @@ def base_bias(shape: MoEShape, seed: int) -> torch.Tensor:
     return (torch.rand(shape.E, generator=g, dtype=torch.float32) * 0.2 - 0.1)
 
 
+def make_tokens(shape: MoEShape, seed: int) -> torch.Tensor:
+    """x [T, d] alone: the token batch of `seed` (the same tensor make_inputs
+    draws for that seed)."""
+    dt = torch_dtype(shape.act_dtype)
+    return torch.randn(shape.T, shape.d, generator=_gen(seed, "x")).to(dt).contiguous()
+
+
 def make_router_inputs(shape: MoEShape, seed: int, beta: Optional[float] = None):
     """x, w_router and bias only (no expert weights)."""
-    dt = torch_dtype(shape.act_dtype)
-    x = torch.randn(shape.T, shape.d, generator=_gen(seed, "x")).to(dt)
+    x = make_tokens(shape, seed)
     w_r = torch.randn(shape.E, shape.d, generator=_gen(seed, "w_router")) * (
         1.0 / shape.d ** 0.5)
     b = base_bias(shape, seed)

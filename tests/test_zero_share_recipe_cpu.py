@@ -23,3 +23,16 @@ def test_recorded_offset_gives_thirty_percent_zero_slots(seed):
     b0[sh.n_routed:] -= float(load_betas()[beta_key(sh, seed)]["beta"])
     _, idx0, _, _ = oracle.route(x[:1024], w_r, b0, sh.top_k)
     assert float(np.mean(idx0 >= sh.n_routed)) < 0.25
+
+
+def test_replica_batches_need_no_tuned_offset():
+    # bench.py gives every rank the model of the base seed and a token batch of
+    # its own seed; the zero-expert offset is tuned per seed for seeds 0-2
+    # only, so the ranks' batches come from make_tokens, which draws x alone
+    import torch
+    from moe_synth import make_tokens
+    sh = get_config("large_e")
+    x7 = make_tokens(sh, 7)
+    assert x7.shape == (sh.T, sh.d) and x7.dtype == torch.bfloat16
+    with pytest.raises(KeyError):
+        make_router_inputs(sh, 7)
