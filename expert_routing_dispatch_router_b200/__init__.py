@@ -111,6 +111,10 @@ def lib():
             "moe_route_noalloc": ([C, P, P, P, P, P, P, P, P], i32),
             "moe_bias_pid_update": ([C, P, P, P, ctypes.POINTER(MoEPIDParams), P], i32),
             "moe_layer_launch_count": ([C], ctypes.c_int32),
+            "moe_ep_local_experts": ([C, ctypes.c_int32, ctypes.c_int32], ctypes.c_int32),
+            "moe_ep_plan": ([C, ctypes.c_int32, ctypes.c_int32, P, P, P, P], i32),
+            "moe_ep_dispatch": ([C, ctypes.c_int32, P, P, P, P, P, P], i32),
+            "moe_ep_return": ([C, ctypes.c_int32, ctypes.c_int32, P, P, P, P, P, P], i32),
             "moe_status_string": ([i32], ctypes.c_char_p),
         }
         for name, (args, res) in sig.items():
@@ -273,6 +277,79 @@ def combine(shape: LayerShape, x, y_perm, topk_idx, topk_gate, slot_row, out=Non
                            _stream(stream))
     _check("moe_combine", st)
     return out
+
+
+def ep_local_experts(shape: LayerShape, rank: int, world: int) -> int:
+    """Routed experts rank `rank` owns when the N routed ids are split evenly
+    over `world` ranks (the first N % world ranks take one more)."""
+    n = int(lib().moe_ep_local_experts(ctypes.byref(shape.c()), rank, world))
+    if n < 0:
+        raise ValueError(f"invalid rank {rank} of {world} or shape {shape}")
+    return n
+
+
+def _pointer_array(tensors, dtype, rows_min, d, device):
+    """Device array of the data addresses of `tensors` (one per rank)."""
+    for r, t in enumerate(tensors):
+        _need(t, f"buffer of rank {r}", dtype)
+        if t.dim() != 2 or t.shape[1] != d or t.shape[0] < rows_min:
+            raise ValueError(f"buffer of rank {r}: shape {tuple(t.shape)}, expected "
+                             f"[>= {rows_min}, {d}]")
+    return torch.tensor([t.data_ptr() for t in tensors], dtype=torch.int64, device=device)
+
+
+def ep_plan(shape: LayerShape, rank: int, world: int, counts_all, stream=None):
+    """-> (dest_row [N], recv_offsets [n_rank + 1]) from every rank's counts
+    (counts_all [world, E] int32, on the device)."""
+    N, E = shape.n_routed, shape.E
+    _need(counts_all, "counts_all", torch.int32, (world, E))
+    dev = counts_all.device
+    dest_row = torch.empty(N, dtype=torch.int32, device=dev)
+    recv_offsets = torch.empty(ep_local_experts(shape, rank, world) + 1, dtype=torch.int32,
+                               device=dev)
+    st = lib().moe_ep_plan(ctypes.byref(shape.c()), rank, world, _ptr(counts_all),
+                           _ptr(dest_row), _ptr(recv_offsets), _stream(stream))
+    _check("moe_ep_plan", st)
+    return dest_row, recv_offsets
+
+
+def ep_dispatch(shape: LayerShape, world: int, x, offsets, row_token, dest_row, recv_bufs,
+                stream=None):
+    """Sends this rank's routed rows into the owners' receive buffers
+    (recv_bufs: one [rows, d] tensor per rank, each with room for every row
+    its experts get)."""
+    T, k, d, N = shape.T, shape.top_k, shape.d, shape.n_routed
+    _need(x, "x", shape.act_dtype, (T, d))
+    _need(offsets, "offsets", torch.int32, (N + 1,))
+    _need(row_token, "row_token", torch.int32, (T * k,))
+    _need(dest_row, "dest_row", torch.int32, (N,))
+    if len(recv_bufs) != world:
+        raise ValueError("one receive buffer per rank")
+    ptrs = _pointer_array(recv_bufs, shape.act_dtype, 0, d, x.device)
+    st = lib().moe_ep_dispatch(ctypes.byref(shape.c()), world, _ptr(x), _ptr(offsets),
+                               _ptr(row_token), _ptr(dest_row), _ptr(ptrs), _stream(stream))
+    _check("moe_ep_dispatch", st)
+    return ptrs  # kept alive by the caller until the stream has run the kernel
+
+
+def ep_return(shape: LayerShape, rank: int, world: int, y_recv, recv_offsets, counts_all,
+              offsets_all, y_homes, stream=None):
+    """Sends this rank's expert output rows back into every source rank's
+    y_perm (y_homes: one [T*k, d] tensor per rank)."""
+    T, k, d, N, E = shape.T, shape.top_k, shape.d, shape.n_routed, shape.E
+    _need(y_recv, "y_recv", shape.act_dtype)
+    _need(recv_offsets, "recv_offsets", torch.int32,
+          (ep_local_experts(shape, rank, world) + 1,))
+    _need(counts_all, "counts_all", torch.int32, (world, E))
+    _need(offsets_all, "offsets_all", torch.int32, (world, N + 1))
+    if len(y_homes) != world:
+        raise ValueError("one y_perm per rank")
+    ptrs = _pointer_array(y_homes, shape.act_dtype, T * k, d, y_recv.device)
+    st = lib().moe_ep_return(ctypes.byref(shape.c()), rank, world, _ptr(y_recv),
+                             _ptr(recv_offsets), _ptr(counts_all), _ptr(offsets_all),
+                             _ptr(ptrs), _stream(stream))
+    _check("moe_ep_return", st)
+    return ptrs
 
 
 def layer_forward(shape: LayerShape, x, w_router, bias, w_gate, w_up, w_down, ws,

@@ -336,6 +336,60 @@ moe_status_t moe_bias_pid_update(const moe_config_t* cfg, const int32_t* counts,
                                      reinterpret_cast<cudaStream_t>(stream)));
 }
 
+int32_t moe_ep_local_experts(const moe_config_t* cfg, int32_t rank, int32_t world) {
+  Shape sh;
+  if (make_shape(cfg, &sh) != MOE_OK || world < 1 || rank < 0 || rank >= world) return -1;
+  return ep_local_experts(rank, (int)sh.N, world);
+}
+
+moe_status_t moe_ep_plan(const moe_config_t* cfg, int32_t rank, int32_t world,
+                         const int32_t* counts_all, int32_t* dest_row, int32_t* recv_offsets,
+                         moe_stream_t stream) {
+  NvtxRange range("moe_ep_plan");
+  Shape sh;
+  moe_status_t s = make_shape(cfg, &sh);
+  if (s != MOE_OK) return s;
+  if (world < 1 || rank < 0 || rank >= world || sh.N < 1) return MOE_ERR_INVALID_ARG;
+  if (!dev_ok(counts_all) || !dev_ok(dest_row) || !dev_ok(recv_offsets))
+    return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_ep_plan(sh, rank, world, counts_all, dest_row, recv_offsets,
+                                    reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_ep_dispatch(const moe_config_t* cfg, int32_t world, const void* x,
+                             const int32_t* offsets, const int32_t* row_token,
+                             const int32_t* dest_row, void* const* recv_x,
+                             moe_stream_t stream) {
+  NvtxRange range("moe_ep_dispatch");
+  Shape sh;
+  moe_status_t s = make_shape(cfg, &sh);
+  if (s != MOE_OK) return s;
+  if (world < 1 || sh.N < 1) return MOE_ERR_INVALID_ARG;
+  if (sh.T == 0) return MOE_OK;  // empty batch: nothing is read or written
+  if (!dev_ok(x) || !dev_ok(offsets) || !dev_ok(row_token) || !dev_ok(dest_row) ||
+      !dev_ok(recv_x))
+    return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_ep_dispatch(sh, world, x, offsets, row_token, dest_row, recv_x,
+                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_ep_return(const moe_config_t* cfg, int32_t rank, int32_t world,
+                           const void* y_recv, const int32_t* recv_offsets,
+                           const int32_t* counts_all, const int32_t* offsets_all,
+                           void* const* y_home, moe_stream_t stream) {
+  NvtxRange range("moe_ep_return");
+  Shape sh;
+  moe_status_t s = make_shape(cfg, &sh);
+  if (s != MOE_OK) return s;
+  if (world < 1 || rank < 0 || rank >= world || sh.N < 1) return MOE_ERR_INVALID_ARG;
+  if (!dev_ok(y_recv) || !dev_ok(recv_offsets) || !dev_ok(counts_all) ||
+      !dev_ok(offsets_all) || !dev_ok(y_home))
+    return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_ep_return(sh, rank, world, y_recv, recv_offsets, counts_all,
+                                      offsets_all, y_home,
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
 moe_status_t moe_selftest_wait_limit(void* ws, size_t ws_bytes, moe_stream_t stream) {
   if (ws == nullptr || ws_bytes < 256 || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
     return MOE_ERR_WORKSPACE;

@@ -114,6 +114,17 @@ int router_launch_count(const Shape& sh);
 bool router_grid_fits(const Shape& sh);
 int router_small_splits(const Shape& sh);
 int expert_ffn_launch_count(const Shape& sh);
+// Expert parallelism over G ranks (csrc/expert_parallel.cu).
+int ep_local_experts(int rank, int N, int G);
+int ep_first_expert(int rank, int N, int G);
+cudaError_t launch_ep_plan(const Shape& sh, int rank, int G, const int32_t* counts_all,
+                           int32_t* dest_row, int32_t* recv_offsets, cudaStream_t st);
+cudaError_t launch_ep_dispatch(const Shape& sh, int G, const void* x, const int32_t* offsets,
+                               const int32_t* row_token, const int32_t* dest_row,
+                               void* const* recv, cudaStream_t st);
+cudaError_t launch_ep_return(const Shape& sh, int rank, int G, const void* y_recv,
+                             const int32_t* recv_offsets, const int32_t* counts_all,
+                             const int32_t* offsets_all, void* const* home, cudaStream_t st);
 cudaError_t launch_bias_pid(const Shape& sh, const int32_t* counts, float* bias,
                             double* state, double target, double kp, double ki,
                             double kd, double max_step, cudaStream_t st);

@@ -36,6 +36,14 @@ One step on rank s (every rank runs the same steps in the same order):
 The functions below compute the plan (split sizes, the regrouping permutation
 and local offsets) from the counts the dispatch step already returns, so the
 plan costs no extra pass over the token rows.
+
+The library's device calls (moe_ep_plan, moe_ep_dispatch, moe_ep_return) do
+the same exchange without the all-to-all and without the regrouping pass:
+once every rank's per-expert counts and offsets are gathered (G x E and
+G x (N + 1) integers), each rank knows where each of its rows lands in its
+owner's receive buffer, already expert-major, and writes it there (peer
+stores on one node); the owners send the expert outputs back the same way.
+`run_ranks_on_one_device` runs that sequence for G ranks on one GPU.
 """
 from __future__ import annotations
 
@@ -187,3 +195,65 @@ def ep_layer_step(rank: int, bounds: Sequence[int], x: torch.Tensor,
             "perm": perm, "local_offsets": local_offsets, "counts": counts.to("cpu"),
             "offsets": offs, "row_token": row_token.to("cpu")}
     return out, plan
+
+
+def run_ranks_on_one_device(shape, xs, w_router, bias, w_gate, w_up, w_down):
+    """Every rank's expert-parallel step with the library's device calls, the
+    ranks run one after another on the current device, each phase one call per
+    rank (so no kernel waits on another). On a node of G GPUs the same calls
+    run one rank per GPU, with the gathers of counts and offsets as
+    collectives, the receive buffers and y_perm as peer memory, and a barrier
+    between the phases.
+
+    shape: the per-rank layer (T tokens per rank); xs: G token batches.
+    Returns (outs, info): every rank's layer output, and the plan and the
+    receive buffers for checks."""
+    import expert_routing_dispatch_router_b200 as moe
+
+    G = len(xs)
+    T, k, d, N, F = shape.T, shape.top_k, shape.d, shape.n_routed, shape.ffn
+    dev = xs[0].device
+    # 1. route and dispatch locally
+    local = []
+    for s in range(G):
+        ws = moe.alloc_workspace(shape, dev)
+        idx, gate = moe.route(shape, xs[s], w_router, bias, ws)
+        counts, offsets, row_token, slot_row, _ = moe.dispatch(shape, xs[s], idx, ws)
+        local.append({"idx": idx, "gate": gate, "counts": counts, "offsets": offsets,
+                      "row_token": row_token, "slot_row": slot_row})
+    # 2. the gathers (a collective on several GPUs)
+    counts_all = torch.stack([p["counts"] for p in local]).contiguous()
+    offsets_all = torch.stack([p["offsets"] for p in local]).contiguous()
+    # 3. plans and the dispatch into the owners' receive buffers
+    cap = G * T * k
+    recv = [torch.zeros(cap, d, dtype=shape.act_dtype, device=dev) for _ in range(G)]
+    recv_offsets, keep = [], []
+    for s in range(G):
+        dest_row, roff = moe.ep_plan(shape, s, G, counts_all)
+        recv_offsets.append(roff)
+        keep.append(moe.ep_dispatch(shape, G, xs[s], local[s]["offsets"],
+                                    local[s]["row_token"], dest_row, recv))
+    # 4. each owner's expert FFN over its receive buffer and its experts
+    y_recv = []
+    lo = 0
+    for r in range(G):
+        n_r = moe.ep_local_experts(shape, r, G)
+        if n_r == 0:
+            y_recv.append(torch.zeros(cap, d, dtype=shape.act_dtype, device=dev))
+            continue
+        sh_r = moe.LayerShape(G * T, d, n_r, shape.n_zero, k, F, shape.act_dtype,
+                              shape.routed_scale)
+        ws_r = moe.alloc_workspace(sh_r, dev)
+        y_recv.append(moe.expert_ffn(sh_r, recv[r], recv_offsets[r], w_gate[lo:lo + n_r],
+                                     w_up[lo:lo + n_r], w_down[lo:lo + n_r], ws_r))
+        lo += n_r
+    # 5. the outputs back to their sources, 6. combine as on one GPU
+    y_perm = [torch.zeros(T * k, d, dtype=shape.act_dtype, device=dev) for _ in range(G)]
+    for r in range(G):
+        keep.append(moe.ep_return(shape, r, G, y_recv[r], recv_offsets[r], counts_all,
+                                  offsets_all, y_perm))
+    outs = [moe.combine(shape, xs[s], y_perm[s], local[s]["idx"], local[s]["gate"],
+                        local[s]["slot_row"]) for s in range(G)]
+    torch.cuda.synchronize(dev)
+    return outs, {"local": local, "counts_all": counts_all, "offsets_all": offsets_all,
+                  "recv": recv, "recv_offsets": recv_offsets, "y_perm": y_perm}

@@ -199,6 +199,59 @@ moe_status_t moe_route_noalloc(const moe_config_t* cfg, const void* x,
                                float* topk_gate, uint8_t* flags,
                                moe_stream_t stream);
 
+/* Expert parallelism across `world` ranks, one GPU each. Ascend deployment
+ * article (10100.com), "Decode节点：EP128超大专家并行" and "多场景模型分层切分优化"
+ * (experts sharded over the cards of a decode instance, DP + EP) and
+ * "底层定制算子深度优化" (Dispatch/Combine operators that support zero experts).
+ * Rank r owns the routed experts [lo_r, lo_r + n_r): an even split of the N
+ * routed ids, the first N % world ranks taking one more (moe_ep_local_experts
+ * gives n_r; lo_r = sum of n_r' over r' < r). Zero experts belong to no rank:
+ * their slots never leave the token's rank. One step on rank s:
+ *  1. moe_route and moe_dispatch on s's own T tokens (counts [E], offsets
+ *     [N+1], row_token; x_perm is not needed);
+ *  2. gather every rank's counts and offsets on every rank (the caller's
+ *     collective): counts_all [world, E] and offsets_all [world, N+1] int32;
+ *  3. moe_ep_plan, then moe_ep_dispatch: s's routed rows go straight into
+ *     their owners' receive buffers, expert-major (expert, source rank,
+ *     source order);
+ *  4. after a barrier, each owner runs moe_expert_ffn on its buffer with the
+ *     recv_offsets of step 3 and its slice of the expert weights (a config
+ *     with n_routed = n_r and T * top_k >= the buffer's rows);
+ *  5. moe_ep_return: each owner sends its output rows back into the sources'
+ *     y_perm, at the rows their dispatches gave them;
+ *  6. after a barrier, moe_combine on each source, as on one GPU.
+ * recv_x and y_home are device arrays of `world` device pointers (the ranks'
+ * receive buffers [rows, d] and y_perm [T*k, d], act_dtype); on one node
+ * these are peer addresses, written with plain stores. A receive buffer
+ * needs room for every row its experts get, at most world * T * top_k.
+ * The calls only order their own work on `stream`: the barriers between the
+ * steps are the caller's. They return MOE_ERR_INVALID_ARG for a bad rank,
+ * world or pointer, and need N >= 1. */
+int32_t moe_ep_local_experts(const moe_config_t* cfg, int32_t rank, int32_t world);
+
+/*  dest_row [N] int32: the first row of rank `rank`'s block of expert e in
+ *  e's owner's receive buffer; recv_offsets [n_rank + 1] int32: rank's own
+ *  receive layout over its experts (the offsets its expert FFN takes). */
+moe_status_t moe_ep_plan(const moe_config_t* cfg, int32_t rank, int32_t world,
+                         const int32_t* counts_all, int32_t* dest_row,
+                         int32_t* recv_offsets, moe_stream_t stream);
+
+/*  Copies x[row_token[j]] for every routed row j < offsets[N] of this rank
+ *  to recv_x[owner(e)] row dest_row[e] + (j - offsets[e]), e the expert of
+ *  row j. */
+moe_status_t moe_ep_dispatch(const moe_config_t* cfg, int32_t world,
+                             const void* x, const int32_t* offsets,
+                             const int32_t* row_token, const int32_t* dest_row,
+                             void* const* recv_x, moe_stream_t stream);
+
+/*  Copies each row i < recv_offsets[n_rank] of y_recv (this rank's expert
+ *  outputs, in its receive order) to y_home[s] row offsets_all[s][e] + its
+ *  order among source s's rows of expert e. */
+moe_status_t moe_ep_return(const moe_config_t* cfg, int32_t rank, int32_t world,
+                           const void* y_recv, const int32_t* recv_offsets,
+                           const int32_t* counts_all, const int32_t* offsets_all,
+                           void* const* y_home, moe_stream_t stream);
+
 /* PID controller on the zero experts' router bias, run between layer calls.
  * "Meituan lancerer LongCat-2.0" (snilld.dk), "MoE i praksis og prisen for
  * fleksibilitet": a PID controller adjusts the router bias so that the

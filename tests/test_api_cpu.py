@@ -173,6 +173,35 @@ def test_route_noalloc_refuses_problems_beyond_its_limits(L):
                                _fake(), None, st) == 2
 
 
+def test_expert_parallel_calls_check_ranks_on_the_host(L):
+    # moe_ep_*: the even split of the routed experts, and refusals of a bad
+    # rank, world or pointer before anything is launched (runs without a GPU)
+    st = P(0)
+    c = cfg(N=7, Z=3, k=3)
+    assert [L.moe_ep_local_experts(ctypes.byref(c), r, 2) for r in range(2)] == [4, 3]
+    assert [L.moe_ep_local_experts(ctypes.byref(c), r, 4) for r in range(4)] == [2, 2, 2, 1]
+    assert [L.moe_ep_local_experts(ctypes.byref(c), r, 9) for r in range(9)] == [1] * 7 + [0] * 2
+    assert L.moe_ep_local_experts(ctypes.byref(c), 2, 2) == -1
+    assert L.moe_ep_local_experts(ctypes.byref(c), 0, 0) == -1
+    f = _fake
+    assert L.moe_ep_plan(ctypes.byref(c), 2, 2, f(), f(), f(), st) == 1  # rank >= world
+    assert L.moe_ep_plan(ctypes.byref(c), -1, 2, f(), f(), f(), st) == 1
+    assert L.moe_ep_plan(ctypes.byref(c), 0, 2, None, f(), f(), st) == 1
+    assert L.moe_ep_dispatch(ctypes.byref(c), 0, f(), f(), f(), f(), f(), st) == 1
+    assert L.moe_ep_dispatch(ctypes.byref(c), 2, f(), f(), f(), f(0x10004), f(), st) == 1
+    assert L.moe_ep_return(ctypes.byref(c), 0, 2, f(), f(), f(), None, f(), st) == 1
+    assert L.moe_ep_return(ctypes.byref(c), 3, 2, f(), f(), f(), f(), f(), st) == 1
+    no_routed = cfg(N=0, Z=4, k=2)
+    assert L.moe_ep_plan(ctypes.byref(no_routed), 0, 2, f(), f(), f(), st) == 1
+    # the split agrees with the host plan's
+    from expert_routing_dispatch_router_b200 import expert_parallel as ep
+    for N, G in ((7, 2), (18, 4), (3, 4), (256, 8), (1, 1)):
+        b = ep.expert_bounds(N, G)
+        cc = cfg(N=N, Z=4, k=2)
+        assert [L.moe_ep_local_experts(ctypes.byref(cc), r, G) for r in range(G)] == \
+            [b[r + 1] - b[r] for r in range(G)]
+
+
 def test_empty_batch_is_a_no_op_before_any_pointer_check(L):
     # T == 0: every entry point returns MOE_OK with all pointers null (empty
     # buffers have no address) and no workspace; nothing is launched, so this
