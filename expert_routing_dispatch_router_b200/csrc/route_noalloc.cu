@@ -11,8 +11,8 @@
 // here in one file-scope device array, kNoAllocScratchFloats floats (16 MiB),
 // which every GPU that loads this library holds until the process exits. The
 // first call on a device, with that device current, looks up the array's
-// device address once (cudaGetSymbolAddress) and remembers it; make that first
-// call before any stream capture on the device. The remembered address belongs
+// device address once (cudaGetSymbolAddress) and remembers it. The remembered
+// address belongs
 // to the device's primary context: after cudaDeviceReset on that device the
 // process must not call this entry point again. Every call on a device shares
 // the one array and leaves the last call's partial sums in it. Nothing has to

@@ -31,8 +31,7 @@
  *    expert outputs y_perm: MOE_F32 (float) or MOE_BF16 (bfloat16).
  *    w_router, bias and topk_gate are always float; indices are int32.
  *  - Every call is asynchronous on `stream` (0 = legacy default stream) and
- *    issues no host synchronisation, so a sequence of calls can be captured
- *    in a CUDA graph.
+ *    issues no host synchronisation.
  *  - Buffers that depend on the routing are sized for the worst case T*top_k
  *    rows, because the number R of routed rows is only known on the device.
  *  - Errors: argument errors are found on the host before anything is
@@ -188,8 +187,7 @@ moe_status_t moe_layer_forward_host(const moe_config_t* cfg, const void* x_host,
  *  CUDA-core router's grid); larger problems return MOE_ERR_UNSUPPORTED
  *  before anything is launched.
  *  The first call on a device (with that device current) looks up the
- *  array's address once; make it before any stream capture on that device.
- *  The address is kept for the life of the process: after cudaDeviceReset
+ *  array's address once. The address is kept for the life of the process: after cudaDeviceReset
  *  on a device, do not call this entry point on it again.
  *  All calls on a device share the array: calls that overlap on the GPU
  *  (other streams or host threads) race and must be ordered by the caller. */
