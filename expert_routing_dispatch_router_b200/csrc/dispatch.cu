@@ -9,8 +9,9 @@
 // Dois Tetos", section "A Primeira Parede").
 //
 // For small batches (the masks of all T tokens fit in shared memory) one block
-// does steps 1-3 in a single launch (dispatch_small_kernel). Otherwise three
-// small kernels plus the gather, no atomics whose order matters:
+// does steps 1-3 in a single launch (dispatch_small_kernel); with at most
+// 2048 routing slots that launch also gathers x_perm. Otherwise three small
+// kernels plus the gather, no atomics whose order matters:
 //  1. dispatch_count_kernel: each block takes 256 tokens and builds, in shared
 //     memory, one 256-bit mask per expert (which of its tokens chose it), then
 //     writes popcount(mask) = the block's count per expert.
@@ -180,18 +181,25 @@ __device__ __forceinline__ int32_t block_exclusive_scan(int32_t v, int32_t* warp
 // Steps 1-3 in one block for a batch whose masks fit in shared memory:
 // mask[e*W + w] bit b = token 32w + b chose e; pre[e*W + w] = set bits of
 // expert e in words before w. rank of token t in expert e = pre + bits below t.
+// With x_perm given (few routing slots), the gather is done in the same
+// launch: every block of the grid repeats steps 1-3 in its own shared memory
+// (the result does not depend on the block), block 0 alone writes them out,
+// and each block copies the token rows of its own run of slots.
 __global__ void __launch_bounds__(1024)
     dispatch_small_kernel(const int32_t* __restrict__ idx, int T, int k, int E, int N,
                           int W, int32_t* __restrict__ counts,
                           int32_t* __restrict__ offsets, int32_t* __restrict__ row_token,
                           int32_t* __restrict__ slot_row, int64_t rows_cap,
                           int32_t* err, int32_t* __restrict__ tile_start, int tile_gu,
-                          int tile_dn) {
+                          int tile_dn, const uint4* __restrict__ x,
+                          uint4* __restrict__ x_perm, int64_t vec_per_row) {
   extern __shared__ uint32_t sm[];
   uint32_t* mask = sm;
   int32_t* pre = reinterpret_cast<int32_t*>(sm + (size_t)E * W);
   int32_t* s_off = pre + (size_t)E * W;
   __shared__ int32_t warp_sums[32];
+  const bool lead = blockIdx.x == 0;  // the block that writes the results
+  if (!lead) err = nullptr;
   griddep_wait();
   griddep_launch_dependents();
   // one thread per routing slot s (token s / k): every slot's expert id is
@@ -218,7 +226,7 @@ __global__ void __launch_bounds__(1024)
       pre[e * W + w] = run;
       run += __popc(mask[e * W + w]);
     }
-    counts[e] = run;
+    if (lead) counts[e] = run;
     if (e < N) s_off[e] = run;
   }
   __syncthreads();
@@ -228,10 +236,42 @@ __global__ void __launch_bounds__(1024)
   __syncthreads();
   if ((int)threadIdx.x < N) {
     s_off[threadIdx.x] = before;
-    offsets[threadIdx.x] = before;
+    if (lead) offsets[threadIdx.x] = before;
   }
-  if (threadIdx.x == 0) offsets[N] = R;
+  if (lead && threadIdx.x == 0) offsets[N] = R;
   __syncthreads();
+  if (x_perm) {
+    // this block's slots [s0, s1), each row cut into `seg` pieces so that
+    // every warp copies about one piece, four 16-byte vectors per lane in
+    // flight
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int per = (Tk + (int)gridDim.x - 1) / (int)gridDim.x;
+    const int s0 = (int)blockIdx.x * per, s1 = min(Tk, s0 + per);
+    const int seg = per >= 32 ? 1 : 32 / per;
+    const int64_t seg_len = (vec_per_row + seg - 1) / seg;
+    for (int item = warp; item < (s1 - s0) * seg; item += 32) {
+      const int s = s0 + item / seg;
+      const int e = idx[s];
+      if (e < 0 || e >= N) continue;
+      const int t = s / k;
+      const int w = t >> 5;
+      const int r = s_off[e] + pre[e * W + w] + __popc(mask[e * W + w] & ((1u << (t & 31)) - 1u));
+      const int64_t q0 = (int64_t)(item % seg) * seg_len;
+      const int64_t q1 = min(vec_per_row, q0 + seg_len);
+      const uint4* src = x + (int64_t)t * vec_per_row;
+      uint4* dst = x_perm + (int64_t)r * vec_per_row;
+      for (int64_t q = q0 + lane; q < q1; q += 4 * 32) {
+        uint4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (q + u * 32 < q1) v[u] = src[q + u * 32];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (q + u * 32 < q1) dst[q + u * 32] = v[u];
+      }
+    }
+  }
+  if (!lead) return;
   if (tile_start) {
     // the expert GEMMs' plans: token-tile prefixes of both GEMMs (v is the
     // count of routed expert threadIdx.x, 0 past N)
@@ -299,8 +339,16 @@ bool dispatch_small_fits(const Shape& sh) {
 
 bool dispatch_plans_tiles(const Shape& sh) { return dispatch_small_fits(sh); }
 
+// Batches of at most this many routing slots gather x_perm inside the
+// one-block dispatch's launch (one warp per slot over the grid).
+constexpr int64_t kSortGatherMaxSlots = 2048;
+
+bool dispatch_gathers_in_sort(const Shape& sh) {
+  return dispatch_small_fits(sh) && sh.T * sh.k <= kSortGatherMaxSlots;
+}
+
 int dispatch_launch_count(const Shape& sh) {
-  return (dispatch_small_fits(sh) ? 1 : 3) + (sh.N > 0 ? 1 : 0);
+  return (dispatch_small_fits(sh) ? 1 : 3) + (sh.N > 0 && !dispatch_gathers_in_sort(sh) ? 1 : 0);
 }
 
 int num_sms() {  // of the current device, cached per device
@@ -332,10 +380,19 @@ cudaError_t launch_dispatch(const Shape& sh, const void* x, const int32_t* idx,
     static std::atomic<uint64_t> attr_set{0};
     e = raise_smem_once(attr_set, dispatch_small_kernel, (int)kSmallDispatchSmem);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(dispatch_small_kernel, dim3(1), dim3(1024), smem, st, idx, (int)sh.T,
+    const bool gather = N > 0 && x_perm && dispatch_gathers_in_sort(sh);
+    const int64_t slots = sh.T * sh.k;
+    // a few slots per block: the redundant sorts run side by side, and the
+    // copies spread over as many SMs
+    int64_t nb = (slots + 3) / 4;
+    if (nb > num_sms()) nb = num_sms();
+    const unsigned blocks = gather ? (unsigned)(nb < 1 ? 1 : nb) : 1u;
+    e = launch_pdl(dispatch_small_kernel, dim3(blocks), dim3(1024), smem, st, idx, (int)sh.T,
                    k, E, N, W, counts, offsets, row_token, slot_row, sh.T * sh.k, err,
-                   tile_start, tile_gu, tile_dn);
+                   tile_start, tile_gu, tile_dn, static_cast<const uint4*>(x),
+                   gather ? static_cast<uint4*>(x_perm) : nullptr, sh.d * sh.es / 16);
     if (e != cudaSuccess) return e;
+    if (gather) return cudaGetLastError();
   } else {
     const size_t smem = (size_t)E * kWords * sizeof(uint32_t);
     const unsigned nch = (unsigned)sh.nchunks;

@@ -419,7 +419,8 @@ int32_t moe_layer_launch_count(const moe_config_t* cfg) {
   if (make_shape(cfg, &sh) != MOE_OK || sh.T == 0) return 0;
   int32_t n = router_launch_count(sh);  // (split + GEMM | logits) + top-k
   n += dispatch_launch_count(sh);  // (count, scan, scatter | small) + gather
-  if (sh.N > 0 && expert_ffn_gathers(sh)) n -= 1;  // the gate/up GEMM gathers
+  if (sh.N > 0 && expert_ffn_gathers(sh) && !dispatch_gathers_in_sort(sh))
+    n -= 1;  // the gate/up GEMM gathers
   n += expert_ffn_launch_count(sh);
   if (sh.N > 0 && expert_ffn_uses_tensor_cores(sh) && dispatch_plans_tiles(sh))
     n -= 1;  // the one-block dispatch writes the GEMM plans

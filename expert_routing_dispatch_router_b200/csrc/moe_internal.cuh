@@ -77,6 +77,8 @@ cudaError_t launch_dispatch(const Shape& sh, const void* x, const int32_t* idx,
                             cudaStream_t st, int32_t* tile_start = nullptr,
                             int tile_gu = 0, int tile_dn = 0);
 bool dispatch_plans_tiles(const Shape& sh);
+// The one-block dispatch also gathers x_perm, in the same launch.
+bool dispatch_gathers_in_sort(const Shape& sh);
 // With x_src and row_token given (the fused layer, where expert_ffn_gathers
 // holds), the gate/up GEMM reads token rows from x by row_token and x_perm is
 // not used.

@@ -84,7 +84,8 @@ def test_cuda_core_router_token_limit(L):
 def test_launch_count(L):
     # router 1 (T <= 256), 2 (CUDA cores) or 3 (split + tensor-core GEMM +
     # top-k); dispatch 1 (one block for T <= 4096) or 3, + gather unless the
-    # single-CTA gate/up GEMM gathers (tensor cores, T <= 1024); FFN 2
+    # single-CTA gate/up GEMM gathers (tensor cores, T <= 1024) or the
+    # one-block dispatch gathers in its own launch (T * k <= 2048); FFN 2
     # (tcgen05, plans written by the one-block dispatch), 3 (tcgen05 + plan)
     # or 2 (CUDA cores), + 1 SwiGLU fixup when a tiny batch splits the gate/up
     # contraction; combine 1
@@ -94,7 +95,9 @@ def test_launch_count(L):
     assert L.moe_layer_launch_count(ctypes.byref(cfg())) == 1 + 1 + 3 + 1
     single = cfg(T=1, d=6144, N=256, Z=64, k=12, F=2048)
     assert L.moe_layer_launch_count(ctypes.byref(single)) == 1 + 1 + 3 + 1
-    assert L.moe_layer_launch_count(ctypes.byref(cfg(dt=moe.MOE_F32))) == 1 + 2 + 2 + 1
+    assert L.moe_layer_launch_count(ctypes.byref(cfg(dt=moe.MOE_F32))) == 1 + 1 + 2 + 1
+    f32_wide = cfg(T=1100, k=2, dt=moe.MOE_F32)  # 2200 slots: a separate gather
+    assert L.moe_layer_launch_count(ctypes.byref(f32_wide)) == 2 + 2 + 2 + 1
     assert L.moe_layer_launch_count(ctypes.byref(cfg(T=300))) == 2 + 1 + 2 + 1
     assert L.moe_layer_launch_count(ctypes.byref(cfg(T=1100))) == 3 + 2 + 2 + 1
     big = cfg(T=16384, d=4096, N=128, Z=32, k=8, F=1024)
