@@ -536,32 +536,35 @@ __global__ void __launch_bounds__(256, 1)
   __threadfence();
   // split sums of the group's tokens into shared memory (the chunks are
   // done): (token, expert) elements spread over the threads, each added in
-  // ascending split order; a thread has the loads of 4 elements x 8 splits in
-  // flight at once
+  // ascending split order; a thread has the loads of 8 elements x 4 splits in
+  // flight at once, so a group of up to 2048 elements takes one round trip
+  // per 4 splits
   float* lgs = reinterpret_cast<float*>(chunks);  // [DG][E]
   const int nz = (int)gridDim.z;
   const int nel = nt * E;
   const int64_t zstride = (int64_t)T * E;
   const float* pbase = part + (int64_t)t0 * E;  // rows t0.. are contiguous
-  for (int el0 = threadIdx.x; el0 < nel; el0 += 4 * blockDim.x) {
-    float sum[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int z0 = 0; z0 < nz; z0 += 8) {
-      float v[4][8];
+  for (int el0 = threadIdx.x; el0 < nel; el0 += 8 * blockDim.x) {
+    float sum[8];
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
+    for (int r = 0; r < 8; ++r) sum[r] = 0.f;
+    for (int z0 = 0; z0 < nz; z0 += 4) {
+      float v[8][4];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
         const int el = el0 + r * (int)blockDim.x;
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
+        for (int q = 0; q < 4; ++q)
           v[r][q] = (el < nel && z0 + q < nz) ? __ldcg(pbase + (z0 + q) * zstride + el) : 0.f;
       }
 #pragma unroll
-      for (int r = 0; r < 4; ++r)
+      for (int r = 0; r < 8; ++r)
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
+        for (int q = 0; q < 4; ++q)
           if (z0 + q < nz) sum[r] += v[r][q];
     }
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
+    for (int r = 0; r < 8; ++r) {
       const int el = el0 + r * (int)blockDim.x;
       if (el < nel) lgs[el] = sum[r];
     }
