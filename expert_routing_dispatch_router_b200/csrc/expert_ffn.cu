@@ -168,6 +168,12 @@ struct GemmArgs {
   // Down GEMM: output rows in bf16 (the expert outputs y_perm) instead of
   // fp32 (the router's logits and split-contraction partials)
   bool out_bf16 = false;
+  // Tensor-core router: when > 0, the A rows are the three bf16 planes of
+  // this many experts, each 32-row quarter of an m-tile holding hi, mid and
+  // lo of 10 experts in rows 3j, 3j + 1, 3j + 2; the epilogue adds the three
+  // planes of an expert (hi + mid, then + lo, in fp32) and writes
+  // out[token][chunk * plane_experts + e]
+  int plane_experts = 0;
 };
 
 struct Unit {
@@ -540,6 +546,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int c = 0; c < 32; ++c)
               if (c0 + c < un.n_valid)
                 outp[(int64_t)(c0 + c) * args.out_cols] = __float2bfloat16_rn(g[c]);
+          } else if (args.plane_experts > 0) {
+            const int64_t e =
+                (int64_t)(un.m % args.mt_chunk) * 40 + (int64_t)ew * 10 + lane / 3;
+            const bool writer = lane < 30 && lane % 3 == 0 && e < args.plane_experts;
+            float* outp = static_cast<float*>(args.out) + (int64_t)un.row0 * args.out_cols +
+                          (int64_t)(un.m / args.mt_chunk) * args.plane_experts + e;
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              const float mid = __shfl_down_sync(0xffffffffu, g[c], 1);
+              const float lo = __shfl_down_sync(0xffffffffu, g[c], 2);
+              if (writer && c0 + c < un.n_valid)
+                outp[(int64_t)(c0 + c) * args.out_cols] = (g[c] + mid) + lo;
+            }
           } else {
             float* outp = static_cast<float*>(args.out) + obase;
 #pragma unroll
@@ -1154,7 +1173,7 @@ cudaError_t launch_simt(const Shape& sh, const void* x_perm, const int32_t* offs
 // tensor cores' fp32 adder runs through. plan is a device int32[4] holding
 // {0, T, 0, ceil(T / kRouterGemmTile)} (the expert's rows, then its token tiles).
 cudaError_t launch_dense_gemm_tc(const void* a, int64_t M, const void* b, int64_t T,
-                                 int64_t K, int kb_chunk, float* out,
+                                 int64_t K, int kb_chunk, int64_t plane_experts, float* out,
                                  const int32_t* plan, int32_t* err, cudaStream_t st) {
   CUtensorMap am, b16, b128;
   if (!make_map(&am, a, (uint64_t)M, (uint64_t)K, BM) ||
@@ -1169,7 +1188,8 @@ cudaError_t launch_dense_gemm_tc(const void* a, int64_t M, const void* b, int64_
   g.err = err;
   g.N = 1;
   g.num_kb = (int)(K / BK);
-  g.out_cols = (int)M * chunks;
+  g.out_cols = (int)(plane_experts > 0 ? plane_experts : M) * chunks;
+  g.plane_experts = (int)plane_experts;
   g.m_tiles = (int)(M / BM) * chunks;
   g.a_rows = (int)M;
   g.mt_chunk = (int)(M / BM);

@@ -38,7 +38,7 @@ WsLayout ws_layout(const Shape& sh) {
   const int splits = router_splits(sh) > router_small_splits(sh) ? router_splits(sh)
                                                                  : router_small_splits(sh);
   size_t part = (size_t)splits * sh.T * sh.E;
-  const size_t tc_part = (size_t)sh.T * router_tc_chunks(sh) * router_planes_rows(sh);
+  const size_t tc_part = (size_t)sh.T * router_tc_chunks(sh) * sh.E;
   if (router_uses_tensor_cores(sh) && tc_part > part) part = tc_part;
   L.logits = take(part * sizeof(float));
   L.planes = take(router_uses_tensor_cores(sh)

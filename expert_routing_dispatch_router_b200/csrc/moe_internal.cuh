@@ -104,11 +104,14 @@ cudaError_t launch_combine(const Shape& sh, const void* x, const void* y_perm,
                            const int32_t* idx, const float* gate,
                            const int32_t* slot_row, void* out, cudaStream_t st,
                            int ysplit = 1);
+// plane_experts > 0: A holds the router's three bf16 planes of that many
+// experts (router_planes_rows layout) and out gets their per-chunk sums,
+// [T][chunks][plane_experts]; otherwise out is [T][chunks][M].
 cudaError_t launch_dense_gemm_tc(const void* a, int64_t M, const void* b, int64_t T,
-                                 int64_t K, int kb_chunk, float* out,
+                                 int64_t K, int kb_chunk, int64_t plane_experts, float* out,
                                  const int32_t* plan, int32_t* err, cudaStream_t st);
 bool router_uses_tensor_cores(const Shape& sh);
-int64_t router_planes_rows(const Shape& sh);   // 3E rounded up to 128
+int64_t router_planes_rows(const Shape& sh);   // 128 per 40 experts
 int router_tc_chunks(const Shape& sh);         // contraction chunks of that router
 int router_launch_count(const Shape& sh);
 // False when the batch is too large for the router path it would take (the

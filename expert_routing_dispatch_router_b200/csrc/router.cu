@@ -579,12 +579,20 @@ __global__ void __launch_bounds__(256, 1)
   if (threadIdx.x == 0) counter[g] = 0;
 }
 
+// Row of plane p (0 hi, 1 mid, 2 lo) of expert e in the tensor-core router's
+// A operand: each 32-row quarter of a 128-row tile holds the three planes of
+// 10 experts side by side (rows 3j, 3j + 1, 3j + 2; rows 30 and 31 are
+// zeros), so the GEMM's epilogue adds an expert's planes inside one warp.
+__host__ __device__ __forceinline__ int64_t plane_row(int64_t e, int p) {
+  return (e / 40) * 128 + ((e % 40) / 10) * 32 + 3 * (e % 10) + p;
+}
+
 // Exact three-way split of the fp32 router weights into bf16 planes for the
 // tensor-core router: hi = bf16(w), mid = bf16(w - hi), lo = bf16(w - hi - mid)
 // (each difference is exact in fp32), so hi + mid + lo carries the 24 bits of
 // w and x . w = x . hi + x . mid + x . lo with x in bf16 and every product
-// exact in fp32. Rows [0,E) of `planes` get hi, [E,2E) mid, [2E,3E) lo, the
-// padding rows up to Ep zeros. Also writes the one-expert plan of the GEMM.
+// exact in fp32. Plane p of expert e goes to row plane_row(e, p); every other
+// row up to Ep is zeros. Also writes the one-expert plan of the GEMM.
 __global__ void __launch_bounds__(256)
     router_split_kernel(const float4* __restrict__ w_r, int64_t E, int64_t d, int64_t Ep,
                         uint2* __restrict__ planes, int32_t* __restrict__ plan,
@@ -595,6 +603,7 @@ __global__ void __launch_bounds__(256)
   const int64_t n = E * q;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
+    const int64_t e = i / q, c4 = i - e * q;
     const float4 w = w_r[i];
     const float v[4] = {w.x, w.y, w.z, w.w};
     uint16_t hb[4], mb[4], lb[4];
@@ -613,13 +622,16 @@ __global__ void __launch_bounds__(256)
       return make_uint2((uint32_t)b[0] | ((uint32_t)b[1] << 16),
                         (uint32_t)b[2] | ((uint32_t)b[3] << 16));
     };
-    planes[i] = pack(hb);
-    planes[n + i] = pack(mb);
-    planes[2 * n + i] = pack(lb);
+    planes[plane_row(e, 0) * q + c4] = pack(hb);
+    planes[plane_row(e, 1) * q + c4] = pack(mb);
+    planes[plane_row(e, 2) * q + c4] = pack(lb);
   }
-  for (int64_t i = 3 * n + (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < Ep * q;
-       i += stride)
-    planes[i] = make_uint2(0u, 0u);
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < Ep * q; i += stride) {
+    const int64_t r = i / q;
+    const int64_t l = r % 32;  // row inside its quarter
+    const int64_t e = (r / 128) * 40 + ((r % 128) / 32) * 10 + l / 3;
+    if (l >= 30 || e >= E) planes[i] = make_uint2(0u, 0u);
+  }
   if (blockIdx.x == 0 && threadIdx.x == 0) {
     plan[0] = 0;
     plan[1] = (int32_t)T;
@@ -635,7 +647,7 @@ __global__ void __launch_bounds__(256)
 // activations use the CUDA-core split-K kernel.
 constexpr int64_t kTcRouterMinTokens = 512;
 
-int64_t router_planes_rows(const Shape& sh) { return (3 * sh.E + 127) / 128 * 128; }
+int64_t router_planes_rows(const Shape& sh) { return (sh.E + 39) / 40 * 128; }
 
 // The tensor-core router restarts its fp32 accumulation every 1024 contraction
 // elements (16 blocks of 64), a chain of 64 MMA steps per partial.
@@ -806,15 +818,15 @@ cudaError_t launch_router(const Shape& sh, const void* x, const float* w_r,
                    reinterpret_cast<const float4*>(w_r), sh.E, sh.d, Ep,
                    static_cast<uint2*>(planes), plan, sh.T, kRouterGemmTile);
     if (e != cudaSuccess) return e;
-    e = launch_dense_gemm_tc(planes, Ep, x, sh.T, sh.d, router_kb_chunk(sh), part, plan,
-                             err, st);
+    e = launch_dense_gemm_tc(planes, Ep, x, sh.T, sh.d, router_kb_chunk(sh), sh.E, part,
+                             plan, err, st);
     if (e != cudaSuccess) return e;
-    // part[t, c * Ep + p * E + e]: chunk c, plane p (hi, mid, lo)
+    // part[t, c * E + e]: chunk c, the three planes already added
     n_outer = router_tc_chunks(sh);
-    outer_stride = Ep;
-    n_inner = 3;
-    inner_stride = sh.E;
-    row_stride = (int64_t)n_outer * Ep;
+    outer_stride = sh.E;
+    n_inner = 1;
+    inner_stride = 0;
+    row_stride = (int64_t)n_outer * sh.E;
   } else {
     const int nsplit = router_splits(sh);
     int64_t kps = (sh.d + nsplit - 1) / nsplit;
