@@ -58,6 +58,9 @@ SHAPES = [
     MoEShape("fz_t512", T=512, d=128, n_routed=6, n_zero=2, top_k=2, ffn=128),
     MoEShape("fz_t1025_pairs", T=1025, d=256, n_routed=4, n_zero=1, top_k=1, ffn=256),
     MoEShape("fz_t4097", T=4097, d=128, n_routed=8, n_zero=2, top_k=2, ffn=128),
+    # tensor-core router with 103 experts: three 40-expert plane tiles, the
+    # last one and its last quarter only partly used
+    MoEShape("fz_t600_e103", T=600, d=256, n_routed=91, n_zero=12, top_k=5, ffn=128),
 ]
 
 
