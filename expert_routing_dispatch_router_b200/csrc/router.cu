@@ -600,37 +600,42 @@ __global__ void __launch_bounds__(256)
   griddep_wait();
   griddep_launch_dependents();
   const int64_t q = d / 4;  // float4 per row
-  const int64_t n = E * q;
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
-    const int64_t e = i / q, c4 = i - e * q;
-    const float4 w = w_r[i];
-    const float v[4] = {w.x, w.y, w.z, w.w};
-    uint16_t hb[4], mb[4], lb[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const __nv_bfloat16 h = __float2bfloat16_rn(v[j]);
-      const float r1 = v[j] - __bfloat162float(h);
-      const __nv_bfloat16 m = __float2bfloat16_rn(r1);
-      const float r2 = r1 - __bfloat162float(m);
-      const __nv_bfloat16 l = __float2bfloat16_rn(r2);
-      hb[j] = __bfloat16_as_ushort(h);
-      mb[j] = __bfloat16_as_ushort(m);
-      lb[j] = __bfloat16_as_ushort(l);
-    }
-    auto pack = [](const uint16_t* b) {
-      return make_uint2((uint32_t)b[0] | ((uint32_t)b[1] << 16),
-                        (uint32_t)b[2] | ((uint32_t)b[3] << 16));
-    };
-    planes[plane_row(e, 0) * q + c4] = pack(hb);
-    planes[plane_row(e, 1) * q + c4] = pack(mb);
-    planes[plane_row(e, 2) * q + c4] = pack(lb);
-  }
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < Ep * q; i += stride) {
-    const int64_t r = i / q;
+  // one row of A per block at a time: expert rows are split, padding rows
+  // (rows 30 and 31 of a quarter, and the unused experts of the last tile)
+  // zeroed
+  for (int64_t r = blockIdx.x; r < Ep; r += gridDim.x) {
     const int64_t l = r % 32;  // row inside its quarter
     const int64_t e = (r / 128) * 40 + ((r % 128) / 32) * 10 + l / 3;
-    if (l >= 30 || e >= E) planes[i] = make_uint2(0u, 0u);
+    if (l >= 30 || e >= E)
+      for (int64_t c4 = threadIdx.x; c4 < q; c4 += blockDim.x)
+        planes[r * q + c4] = make_uint2(0u, 0u);
+  }
+  for (int64_t e = blockIdx.x; e < E; e += gridDim.x) {
+    const int64_t hi_row = plane_row(e, 0) * q, mid_row = plane_row(e, 1) * q,
+                  lo_row = plane_row(e, 2) * q;
+    for (int64_t c4 = threadIdx.x; c4 < q; c4 += blockDim.x) {
+      const float4 w = w_r[e * q + c4];
+      const float v[4] = {w.x, w.y, w.z, w.w};
+      uint16_t hb[4], mb[4], lb[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const __nv_bfloat16 h = __float2bfloat16_rn(v[j]);
+        const float r1 = v[j] - __bfloat162float(h);
+        const __nv_bfloat16 m = __float2bfloat16_rn(r1);
+        const float r2 = r1 - __bfloat162float(m);
+        const __nv_bfloat16 l = __float2bfloat16_rn(r2);
+        hb[j] = __bfloat16_as_ushort(h);
+        mb[j] = __bfloat16_as_ushort(m);
+        lb[j] = __bfloat16_as_ushort(l);
+      }
+      auto pack = [](const uint16_t* b) {
+        return make_uint2((uint32_t)b[0] | ((uint32_t)b[1] << 16),
+                          (uint32_t)b[2] | ((uint32_t)b[3] << 16));
+      };
+      planes[hi_row + c4] = pack(hb);
+      planes[mid_row + c4] = pack(mb);
+      planes[lo_row + c4] = pack(lb);
+    }
   }
   if (blockIdx.x == 0 && threadIdx.x == 0) {
     plan[0] = 0;
@@ -811,8 +816,7 @@ cudaError_t launch_router(const Shape& sh, const void* x, const float* w_r,
   }
   if (router_uses_tensor_cores(sh)) {
     const int64_t Ep = router_planes_rows(sh);
-    const int64_t n4 = sh.E * sh.d / 4;
-    int64_t blocks = (n4 + 255) / 256;
+    int64_t blocks = Ep;  // rows of the planes, one block per row at a time
     if (blocks > 4 * num_sms()) blocks = 4 * num_sms();
     e = launch_pdl(router_split_kernel, dim3((unsigned)blocks), dim3(256), 0, st,
                    reinterpret_cast<const float4*>(w_r), sh.E, sh.d, Ep,
