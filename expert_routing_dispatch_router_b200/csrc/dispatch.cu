@@ -84,12 +84,22 @@ __global__ void __launch_bounds__(1024)
   __shared__ int32_t total_s;
   griddep_wait();
   griddep_launch_dependents();
+  // per expert, the exclusive scan over the blocks' counts; the counts of 16
+  // blocks are loaded before any of them is overwritten, so a scan over many
+  // blocks takes one memory round trip per 16 of them
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     int32_t run = 0;
-    for (int64_t c = 0; c < nchunks; ++c) {
-      const int32_t v = chunk_base[c * E + e];
-      chunk_base[c * E + e] = run;
-      run += v;
+    for (int64_t c0 = 0; c0 < nchunks; c0 += 16) {
+      int32_t v[16];
+#pragma unroll
+      for (int q = 0; q < 16; ++q)
+        v[q] = c0 + q < nchunks ? chunk_base[(c0 + q) * E + e] : 0;
+#pragma unroll
+      for (int q = 0; q < 16; ++q)
+        if (c0 + q < nchunks) {
+          chunk_base[(c0 + q) * E + e] = run;
+          run += v[q];
+        }
     }
     counts[e] = run;
   }
