@@ -2,7 +2,7 @@
 moe_ep_dispatch, moe_ep_return), with G ranks run one after another on one
 GPU, each phase one call per rank: no kernel waits on another.
 
-Checks, for G = 2 and 4 and an uneven split of the experts:
+Checks, for G = 2, 4 and 8 and an uneven split of the experts:
   * every rank's layer output matches the oracle's per-token layer on that
     rank's tokens, within the layer tolerance;
   * each owner's receive buffer holds, bit for bit, the token rows of its
@@ -33,6 +33,8 @@ CASES = [
     # more ranks than some experts need: 3 experts over 4 ranks, f32 (CUDA cores)
     (MoEShape("ep4_f32", T=40, d=128, n_routed=3, n_zero=3, top_k=2, ffn=64,
               act_dtype="f32"), 4),
+    # one 8-GPU node's worth of ranks: 37 experts (5 x 5 + 4 x 3), top-6
+    (MoEShape("ep8", T=64, d=256, n_routed=37, n_zero=8, top_k=6, ffn=128), 8),
 ]
 
 
